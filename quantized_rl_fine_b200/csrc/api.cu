@@ -1,0 +1,411 @@
+// C ABI of libmoeq: argument validation, workspace layout, tensor maps and
+// kernel launches. Built as one translation unit together with the kernel
+// sources (see moeq_all.cu).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "dequant.cuh"
+#include "gemm.cuh"
+#include "launchers.cuh"
+
+namespace moeq {
+
+
+namespace {
+
+// --------------------------------------------------------------- test hook kernel
+
+// One thread per (row, group): 32 elements of a row from its 16 packed bytes
+// and its group scale, with the GEMM kernels' dequant functions.
+template <int FMT>
+__global__ void dequant_rows_kernel(const uint8_t* __restrict__ packed, const void* __restrict__ scales,
+                                    int64_t R, int K, uint16_t* __restrict__ out) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int G = K / 32;
+  if (gid >= R * G) return;
+  const int64_t r = gid / G;
+  const int g = static_cast<int>(gid % G);
+  const uint4 pk = *reinterpret_cast<const uint4*>(packed + r * (K / 2) + g * 16);
+  uint32_t sbits;
+  if constexpr (FMT == MOE_W_INT4_G32_BF16) {
+    sbits = static_cast<const uint16_t*>(scales)[static_cast<int64_t>(g) * R + r];
+  } else {
+    sbits = static_cast<const uint8_t*>(scales)[static_cast<int64_t>(g) * R + r];
+  }
+  uint32_t o[16];
+  dequant32<FMT>(pk, sbits, o);
+  uint4* dst = reinterpret_cast<uint4*>(out + r * K + g * 32);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+}
+
+// --------------------------------------------------------------- host helpers
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D tiled tensor map over a row-major [rows][cols] array.
+bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize,
+                 uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+                 CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+int max_smem_optin() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 227 * 1024;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 227 * 1024;
+  return n;
+}
+
+// Token rows per tile from the mean rows per expert: ~1.4x the mean split
+// into as few tiles of <= 256 as possible, rounded up to a multiple of 16.
+int choose_bn(int64_t M, int E) {
+  if (const char* env = getenv("MOEQ_BN")) {
+    const int v = atoi(env);
+    if (v >= 16 && v <= 256 && v % 16 == 0) return v;
+  }
+  const double mean = static_cast<double>(M) / std::max(1, E);
+  const double want = std::max(1.0, 1.4 * mean);
+  const int tiles = static_cast<int>((want + 255.0) / 256.0);
+  int bn = static_cast<int>((want / tiles + 15.0) / 16.0) * 16;
+  return std::min(256, std::max(16, bn));
+}
+
+int next_pow2(int x) {
+  int p = 32;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+moe_status check_qweight(const moe_qweight* w) {
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (!w->packed || !w->scales) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w->packed) || !aligned16(w->scales)) return MOE_ERR_MISALIGNED;
+  if (w->fmt != MOE_W_INT4_G32_BF16 && w->fmt != MOE_W_MXFP4_G32_E8M0) return MOE_ERR_INVALID_ARG;
+  if (w->E < 1 || w->E > 1024 || w->N < 1 || w->K < 1) return MOE_ERR_INVALID_ARG;
+  if (w->K % 64 != 0 || w->N % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(w->E) * w->N >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_groups(const moe_groups* g, int E) {
+  if (!g || !g->expert_offsets || !g->active || !g->num_active) return MOE_ERR_INVALID_ARG;
+  if (g->E != E) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+struct GemmPlan {
+  int BN, stages, grid, n_ftiles;
+  uint32_t stage_bytes;
+  size_t smem;
+  size_t sched_bytes;
+};
+
+// F: output features; tile_f: output features per tile (128, or 64 for the
+// SwiGLU forward, whose tile holds 64 gate and the 64 matching up rows).
+GemmPlan plan_gemm(int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
+  GemmPlan pl;
+  pl.BN = choose_bn(M, w->E);
+  pl.stage_bytes = gemm_stage_bytes(pl.BN, fmt);
+  const int avail = max_smem_optin();
+  int stages = 8;
+  while (stages > 2 && static_cast<int>(stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages)) > avail)
+    --stages;
+  pl.stages = stages;
+  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages);
+  pl.n_ftiles = (F + tile_f - 1) / tile_f;
+  const int64_t bound = static_cast<int64_t>(pl.n_ftiles) *
+                        (std::min<int64_t>(w->E, M) + (M + pl.BN - 1) / pl.BN);
+  pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound)));
+  pl.sched_bytes = align_up(static_cast<size_t>(w->E + 3) * sizeof(int32_t), 256);
+  return pl;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Runs one grouped GEMM launch (schedule + main kernel) on `a_or_dout` rows.
+moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qweight* w,
+                    const moe_groups* g, void* out, int64_t ldo, void* saved, int32_t* sched,
+                    const GemmPlan& pl, cudaStream_t s) {
+  const int F = (mode == kModeFwd) ? (epi == MOE_EPI_SWIGLU ? w->N / 2 : w->N) : w->K;
+  const int R = (mode == kModeFwd) ? w->K : w->N;
+  CUtensorMap tb, tw, ts;
+  const bool int4 = w->fmt == MOE_W_INT4_G32_BF16;
+  if (!make_map_2d(&tb, bmat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, 64, pl.BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return MOE_ERR_CUDA;
+  if (mode == kModeFwd) {
+    if (!make_map_2d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K / 2,
+                     static_cast<uint64_t>(w->E) * w->N, 32, 64, CU_TENSOR_MAP_SWIZZLE_32B))
+      return MOE_ERR_CUDA;
+    if (!make_map_2d(&ts, w->scales,
+                     int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                     int4 ? 2 : 1, w->N, static_cast<uint64_t>(w->E) * (w->K / 32), 64, 2,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MOE_ERR_CUDA;
+  } else {
+    if (!make_map_2d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K / 2,
+                     static_cast<uint64_t>(w->E) * w->N, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B))
+      return MOE_ERR_CUDA;
+    if (!make_map_2d(&ts, w->scales,
+                     int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                     int4 ? 2 : 1, w->N, static_cast<uint64_t>(w->E) * (w->K / 32), 64, 4,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MOE_ERR_CUDA;
+  }
+  cudaError_t e = launch_build_schedule(g->expert_offsets, g->active, g->num_active, sched, w->E,
+                                        static_cast<int>(M), pl.BN, pl.n_ftiles, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  GemmArgs p;
+  p.offsets = g->expert_offsets;
+  p.active = g->active;
+  p.sched = sched;
+  p.E = w->E;
+  p.N = w->N;
+  p.K = w->K;
+  p.M = static_cast<int32_t>(M);
+  p.BN = pl.BN;
+  p.acc_cols = (pl.BN + 31) / 32 * 32;
+  p.tmem_cols = next_pow2(2 * p.acc_cols);
+  p.F = F;
+  p.R = R;
+  p.stages = pl.stages;
+  p.stage_bytes = pl.stage_bytes;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.ldo = ldo;
+  p.saved = static_cast<__nv_bfloat16*>(saved);
+  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, tb, tw, ts, p, pl.grid, pl.smem, s));
+}
+
+}  // namespace
+}  // namespace moeq
+
+using namespace moeq;
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOEQ_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_MISALIGNED: return "MOE_ERR_MISALIGNED";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int32_t E, int32_t k,
+                             int64_t d, int32_t chunk_size, int32_t* topk_idx, float* gates,
+                             int32_t* expert_offsets, int32_t* active, int32_t* num_active,
+                             int32_t* chunk_offsets, int32_t* num_chunks, int32_t* perm_token,
+                             int32_t* inv_perm, void* x_perm, void* ws, size_t* ws_bytes,
+                             void* stream) {
+  if (!ws_bytes) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || chunk_size < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  const int nblk = route_num_blocks(T);
+  const size_t need = align_up(static_cast<size_t>(nblk) * E * sizeof(int32_t), 256);
+  if (!ws) {
+    *ws_bytes = need;
+    return MOE_OK;
+  }
+  if (*ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  const void* ptrs[] = {logits, topk_idx, gates, expert_offsets, active, num_active,
+                        chunk_offsets, num_chunks, perm_token, inv_perm};
+  for (const void* p : ptrs) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  if (x) {
+    if (!x_perm || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_MISALIGNED;
+  }
+  return cuda_status(launch_route(logits, x, static_cast<int>(T), E, k, d, chunk_size, topk_idx,
+                                  gates, expert_offsets, active, num_active, chunk_offsets,
+                                  num_chunks, perm_token, inv_perm, x ? x_perm : nullptr,
+                                  static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
+                                 const moe_groups* g, const void* adapter, int32_t epi, void* out,
+                                 void* saved_gu, void* ws, size_t* ws_bytes, void* stream) {
+  if (!ws_bytes) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_qweight(w);
+  if (st != MOE_OK) return st;
+  if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  if (epi != MOE_EPI_NONE && epi != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (epi == MOE_EPI_SWIGLU && w->N % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  const int F = (epi == MOE_EPI_SWIGLU) ? w->N / 2 : w->N;
+  const GemmPlan pl = plan_gemm(M, w, F, epi == MOE_EPI_SWIGLU ? 64 : 128, w->fmt);
+  const size_t xa_bytes = adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
+  const size_t need = pl.sched_bytes + xa_bytes;
+  if (!ws) {
+    *ws_bytes = need;
+    return MOE_OK;
+  }
+  if (*ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  if ((st = check_groups(g, w->E)) != MOE_OK) return st;
+  if (!a || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(out) || (saved_gu && !aligned16(saved_gu)) ||
+      (adapter && !aligned16(adapter)))
+    return MOE_ERR_MISALIGNED;
+  if (saved_gu && epi != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* sched = static_cast<int32_t*>(ws);
+  const void* bmat = a;
+  if (adapter) {
+    void* xa = static_cast<uint8_t*>(ws) + pl.sched_bytes;
+    cudaError_t e = launch_adapter_apply(a, adapter, g->expert_offsets, w->E, static_cast<int>(M),
+                                         w->K, xa, false, s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    bmat = xa;
+  }
+  return run_gemm(kModeFwd, epi, bmat, M, w, g, out, F, saved_gu, sched, pl, s);
+}
+
+moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweight* w,
+                                    const moe_groups* g, int32_t epi, const void* saved_gu,
+                                    const void* adapter, const void* a, void* din,
+                                    float* d_adapter, void* ws, size_t* ws_bytes, void* stream) {
+  if (!ws_bytes) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_qweight(w);
+  if (st != MOE_OK) return st;
+  if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
+  if (epi != MOE_EPI_NONE && epi != MOE_EPI_SWIGLU_BWD) return MOE_ERR_INVALID_ARG;
+  const bool with_adapter = adapter != nullptr;
+  if (with_adapter && (epi != MOE_EPI_NONE || !a || !d_adapter)) return MOE_ERR_INVALID_ARG;
+  if (!with_adapter && (a || d_adapter)) return MOE_ERR_INVALID_ARG;
+  if (epi == MOE_EPI_SWIGLU_BWD && !saved_gu) return MOE_ERR_INVALID_ARG;
+  const GemmPlan pl = plan_gemm(M, w, w->K, 128, w->fmt);
+  const size_t dx_bytes = with_adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
+  const size_t need = pl.sched_bytes + dx_bytes;
+  if (!ws) {
+    *ws_bytes = need;
+    return MOE_OK;
+  }
+  if (*ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  if ((st = check_groups(g, w->E)) != MOE_OK) return st;
+  if (!dout || !din) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(din) || (saved_gu && !aligned16(saved_gu)) ||
+      (adapter && !aligned16(adapter)) || (a && !aligned16(a)) ||
+      (d_adapter && !aligned16(d_adapter)))
+    return MOE_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* sched = static_cast<int32_t*>(ws);
+  if (epi == MOE_EPI_SWIGLU_BWD) {
+    return run_gemm(kModeBwd, epi, dout, M, w, g, din, 2 * static_cast<int64_t>(w->K),
+                    const_cast<void*>(saved_gu), sched, pl, s);
+  }
+  if (!with_adapter) {
+    return run_gemm(kModeBwd, epi, dout, M, w, g, din, w->K, nullptr, sched, pl, s);
+  }
+  void* dxa = static_cast<uint8_t*>(ws) + pl.sched_bytes;
+  st = run_gemm(kModeBwd, epi, dout, M, w, g, dxa, w->K, nullptr, sched, pl, s);
+  if (st != MOE_OK) return st;
+  cudaError_t e = launch_adapter_apply(dxa, adapter, g->expert_offsets, w->E, static_cast<int>(M),
+                                       w->K, din, true, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_status(launch_adapter_grad(a, dxa, g->expert_offsets, w->E, w->K, d_adapter, s));
+}
+
+moe_status moe_unpermute_combine(const void* rows, const int32_t* inv_perm, const float* gates,
+                                 int64_t T, int32_t k, int64_t D, void* out, int32_t mode,
+                                 void* stream) {
+  if (!rows || !inv_perm || !out) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || k < 1 || k > 32 || D < 8 || D % 8 != 0 || (mode != 0 && mode != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(rows) || !aligned16(inv_perm) || !aligned16(out) || (gates && !aligned16(gates)))
+    return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_combine(rows, inv_perm, gates, static_cast<int>(T), k, D, out, mode,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_get_device_error(int32_t* code, void* stream) {
+  if (!code) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int32_t zero = 0;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
+  *code = v;
+  return MOE_OK;
+}
+
+moe_status moe_test_dequant(const void* packed, const void* scales, int64_t R, int32_t K,
+                            int32_t fmt, void* out, void* stream) {
+  if (!packed || !scales || !out || R < 1 || K < 64 || K % 64 != 0) return MOE_ERR_INVALID_ARG;
+  if (fmt != MOE_W_INT4_G32_BF16 && fmt != MOE_W_MXFP4_G32_E8M0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(packed) || !aligned16(scales) || !aligned16(out)) return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_dequant_rows(packed, scales, R, K, fmt, out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_test_set_wait_budget(int64_t cycles) {
+  const long long v = cycles > 0 ? static_cast<long long>(cycles) : kDefaultWaitBudget;
+  return cuda_status(cudaMemcpyToSymbol(g_wait_budget, &v, sizeof(v)));
+}
+
+}  // extern "C"
+
+namespace moeq {
+
+cudaError_t launch_dequant_rows(const void* packed, const void* scales, int64_t R, int K, int fmt,
+                                void* out, cudaStream_t s) {
+  const int64_t n = R * (K / 32);
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  if (fmt == MOE_W_INT4_G32_BF16)
+    dequant_rows_kernel<MOE_W_INT4_G32_BF16><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+        static_cast<const uint8_t*>(packed), scales, R, K, static_cast<uint16_t*>(out));
+  else
+    dequant_rows_kernel<MOE_W_MXFP4_G32_E8M0><<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+        static_cast<const uint8_t*>(packed), scales, R, K, static_cast<uint16_t*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moeq

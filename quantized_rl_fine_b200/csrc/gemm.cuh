@@ -1,0 +1,42 @@
+// Host-side interface of the grouped low-bit GEMM kernels (internal).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moeq {
+
+constexpr int kModeFwd = 0;   // D[f, t] = sum_k W[e][f][k] a[t][k]
+constexpr int kModeBwd = 1;   // D[f, t] = sum_n W[e][n][f] dout[t][n]
+
+struct GemmArgs {
+  const int32_t* offsets;     // [E+1] expert row offsets
+  const int32_t* active;      // [E] active experts (ascending)
+  const int32_t* sched;       // [E+3]: {A, total tiles, tile_start[0..A]}
+  int32_t E, N, K;            // weight stack dims, W[e] is [N][K]
+  int32_t M;                  // rows of a / dout / out
+  int32_t BN;                 // token rows per tile (multiple of 16, <= 256)
+  int32_t acc_cols;           // TMEM columns per accumulator buffer (>= BN, multiple of 32)
+  int32_t tmem_cols;          // TMEM columns allocated (power of two, >= 2 * acc_cols)
+  int32_t F;                  // output features (fwd: N or N/2 with SwiGLU; bwd: K)
+  int32_t R;                  // reduction length (fwd: K; bwd: N)
+  int32_t stages;             // pipeline depth
+  uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
+  __nv_bfloat16* out;         // [M][ldo]
+  int64_t ldo;
+  __nv_bfloat16* saved;       // fwd SwiGLU: written [M][N]; bwd SwiGLU: read [M][2K]
+};
+
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& tb,
+                                 const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
+                                 int grid, size_t smem, cudaStream_t s);
+cudaError_t launch_build_schedule(const int32_t* offsets, const int32_t* active,
+                                  const int32_t* num_active, int32_t* sched, int E, int M, int BN,
+                                  int n_ftiles, cudaStream_t s);
+uint32_t gemm_stage_bytes(int BN, int fmt);
+uint32_t gemm_fixed_smem_bytes(int stages);
+constexpr int kGemmThreads = 384;
+
+}  // namespace moeq

@@ -1,0 +1,24 @@
+// Host launchers of the non-GEMM kernels (internal to libmoeq).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moeq {
+
+int route_num_blocks(int64_t T);
+cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k, int64_t d,
+                         int chunk_size, int32_t* topk_idx, float* gates, int32_t* offsets,
+                         int32_t* active, int32_t* num_active, int32_t* chunk_offsets,
+                         int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
+                         void* x_perm, int32_t* block_counts, cudaStream_t s);
+cudaError_t launch_combine(const void* rows, const int32_t* inv_perm, const float* gates, int T,
+                           int k, int64_t D, void* out, int mode, cudaStream_t s);
+cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* offsets, int E,
+                                 int M, int K, void* out, bool transpose, cudaStream_t s);
+cudaError_t launch_adapter_grad(const void* x, const void* dxp, const int32_t* offsets, int E,
+                                int K, float* dR, cudaStream_t s);
+cudaError_t launch_dequant_rows(const void* packed, const void* scales, int64_t R, int K, int fmt,
+                                void* out, cudaStream_t s);
+
+}  // namespace moeq

@@ -1,0 +1,239 @@
+// Router top-k -> per-expert groups -> active-expert chunks -> stable
+// permutation of the token rows.
+//
+// Orbit article, "Active-expert-chunked dequantization": each token only
+// activates the experts its router selects, and the selected experts are
+// batched into fixed-size groups before the grouped GEMM.
+//
+// Three kernels, no host round trip:
+//  1. route_topk_kernel: one warp per token (8 tokens per warp, 64 per
+//     block); k rounds of a warp-wide argmax (ties to the lower expert id),
+//     softmax of the k selected logits, and a per-block expert histogram in
+//     shared memory.
+//  2. route_scan_kernel: one block; per expert, an exclusive scan of the
+//     block histograms (block bases for step 3), then scans over experts for
+//     the offsets, the active list and the chunk table.
+//  3. route_scatter_kernel: per block, a 64-bit token mask per expert built
+//     with shared-memory atomicOr; the rank of token t inside expert e is the
+//     popcount of the mask below t, which gives the stable position
+//     offsets[e] + block_base[e] + rank. The same block copies the token rows
+//     to their permuted positions with 16-byte loads and stores.
+#include "common.cuh"
+#include "launchers.cuh"
+
+namespace moeq {
+
+namespace {
+
+constexpr int kRouteTokensPerBlock = 64;
+constexpr int kRouteThreads = 256;
+
+__device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                  int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+                  int32_t* __restrict__ block_counts) {
+  extern __shared__ int32_t hist[];   // [E]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per_warp = kRouteTokensPerBlock / (kRouteThreads / 32);
+  const int nper = (E + 31) / 32;     // logits per lane (<= 32)
+  for (int u = 0; u < per_warp; ++u) {
+    const int t = blockIdx.x * kRouteTokensPerBlock + warp * per_warp + u;
+    if (t >= T) break;
+    const float* row = logits + static_cast<int64_t>(t) * E;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int e = lane + 32 * i;
+      v[i] = (i < nper && e < E) ? row[e] : 0.0f;
+    }
+    uint32_t taken = 0;
+    float my_val = 0.0f;
+    int my_idx = 0;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int e = lane + 32 * i;
+        if (i < nper && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
+          bv = v[i];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == j) {
+        my_val = bv;
+        my_idx = bi;
+      }
+    }
+    // gates: softmax over the k selected logits (the first is the largest)
+    const float top = __shfl_sync(0xffffffffu, my_val, 0);
+    const float z = (lane < k) ? expf(my_val - top) : 0.0f;
+    float sum = z;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < k) {
+      topk_idx[static_cast<int64_t>(t) * k + lane] = my_idx;
+      gates[static_cast<int64_t>(t) * k + lane] = z / sum;
+      atomicAdd(&hist[my_idx], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
+}
+
+// One block of 1024 threads, E <= 1024.
+__global__ void __launch_bounds__(1024)
+route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk_size,
+                  int32_t* __restrict__ offsets, int32_t* __restrict__ active,
+                  int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
+                  int32_t* __restrict__ num_chunks) {
+  __shared__ int32_t ws_cnt[32];
+  __shared__ int32_t ws_act[32];
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int64_t i = static_cast<int64_t>(b) * E + e;
+      const int c = block_counts[i];
+      block_counts[i] = cnt;      // becomes the block's base inside expert e
+      cnt += c;
+    }
+  }
+  const int act = (e < E && cnt > 0) ? 1 : 0;
+  const int lane = e & 31, w = e >> 5;
+  int xc = cnt, xa = act;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int yc = __shfl_up_sync(0xffffffffu, xc, o);
+    const int ya = __shfl_up_sync(0xffffffffu, xa, o);
+    if (lane >= o) {
+      xc += yc;
+      xa += ya;
+    }
+  }
+  if (lane == 31) {
+    ws_cnt[w] = xc;
+    ws_act[w] = xa;
+  }
+  __syncthreads();
+  if (w == 0) {
+    int sc = ws_cnt[lane], sa = ws_act[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yc = __shfl_up_sync(0xffffffffu, sc, o);
+      const int ya = __shfl_up_sync(0xffffffffu, sa, o);
+      if (lane >= o) {
+        sc += yc;
+        sa += ya;
+      }
+    }
+    ws_cnt[lane] = sc;
+    ws_act[lane] = sa;
+  }
+  __syncthreads();
+  const int incl_c = xc + (w > 0 ? ws_cnt[w - 1] : 0);
+  const int incl_a = xa + (w > 0 ? ws_act[w - 1] : 0);
+  if (e < E) {
+    offsets[e] = incl_c - cnt;
+    if (act) active[incl_a - 1] = e;
+  }
+  if (e == E - 1) offsets[E] = incl_c;
+  __syncthreads();
+  const int A = ws_act[(E - 1) >> 5] ;   // inclusive total of the last warp holding an expert
+  const int nch = (A + chunk_size - 1) / chunk_size;
+  if (e == 0) {
+    *num_active = A;
+    *num_chunks = nch;
+  }
+  for (int c = e; c <= nch; c += blockDim.x) chunk_offsets[c] = min(c * chunk_size, A);
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ block_base,
+                     const int32_t* __restrict__ offsets, int T, int E, int k,
+                     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm,
+                     const uint4* __restrict__ x, uint4* __restrict__ x_perm, int64_t row_vec) {
+  extern __shared__ uint32_t sm[];      // lo[E], hi[E], pos[64 * k]
+  uint32_t* lo = sm;
+  uint32_t* hi = sm + E;
+  int32_t* pos = reinterpret_cast<int32_t*>(sm + 2 * E);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    lo[e] = 0;
+    hi[e] = 0;
+  }
+  __syncthreads();
+  const int t0 = blockIdx.x * kRouteTokensPerBlock;
+  const int ntok = min(kRouteTokensPerBlock, T - t0);
+  const int nent = ntok * k;
+  for (int i = threadIdx.x; i < nent; i += blockDim.x) {
+    const int tl = i / k;
+    const int e = topk_idx[static_cast<int64_t>(t0) * k + i];
+    atomicOr(tl < 32 ? &lo[e] : &hi[e], 1u << (tl & 31));
+  }
+  __syncthreads();
+  const int32_t* base = block_base + static_cast<int64_t>(blockIdx.x) * E;
+  for (int i = threadIdx.x; i < nent; i += blockDim.x) {
+    const int tl = i / k;
+    const int e = topk_idx[static_cast<int64_t>(t0) * k + i];
+    const int rank = (tl < 32) ? __popc(lo[e] & ((1u << tl) - 1u))
+                               : __popc(lo[e]) + __popc(hi[e] & ((1u << (tl - 32)) - 1u));
+    const int p = offsets[e] + base[e] + rank;
+    perm_token[p] = t0 + tl;
+    inv_perm[static_cast<int64_t>(t0) * k + i] = p;
+    pos[i] = p;
+  }
+  if (x == nullptr) return;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < nent; i += kRouteThreads / 32) {
+    const uint4* src = x + static_cast<int64_t>(t0 + i / k) * row_vec;
+    uint4* dst = x_perm + static_cast<int64_t>(pos[i]) * row_vec;
+    for (int64_t c = lane; c < row_vec; c += 32) dst[c] = src[c];
+  }
+}
+
+}  // namespace
+
+int route_num_blocks(int64_t T) {
+  return static_cast<int>((T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock);
+}
+
+cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k, int64_t d,
+                         int chunk_size, int32_t* topk_idx, float* gates, int32_t* offsets,
+                         int32_t* active, int32_t* num_active, int32_t* chunk_offsets,
+                         int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
+                         void* x_perm, int32_t* block_counts, cudaStream_t s) {
+  const int nblk = route_num_blocks(T);
+  route_topk_kernel<<<nblk, kRouteThreads, E * sizeof(int32_t), s>>>(logits, T, E, k, topk_idx,
+                                                                     gates, block_counts);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, chunk_size, offsets, active,
+                                       num_active, chunk_offsets, num_chunks);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t sm = (2 * E + kRouteTokensPerBlock * k) * sizeof(uint32_t);
+  route_scatter_kernel<<<nblk, kRouteThreads, sm, s>>>(
+      topk_idx, block_counts, offsets, T, E, k, perm_token, inv_perm,
+      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), d / 8);
+  return cudaGetLastError();
+}
+
+}  // namespace moeq

@@ -1,0 +1,257 @@
+"""Parity of the CUDA library (through the C ABI) with the CPU oracle.
+
+Bit-exact: dequantized weights, top-k indices, offsets, active list, chunk
+table, permutation and permuted rows. BF16 outputs that end the computation:
+max-abs <= 2e-2 and rel-L2 <= 5e-3 against the oracle (the workload's
+criterion); per-slot intermediates: |err| <= 2e-2 + one BF16 ulp.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from quantized_rl_fine_b200 import layer, moeq, synth
+from quantized_rl_fine_b200.configs import MXFP4_UP, TINY_INT4, MoEConfig
+
+from _common import (assert_close_final, assert_close_intermediate, bf16_bits, f64,
+                     oracle_qweight)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+TINY_TRAIN = MoEConfig("tiny_train_int4_adapter", E=8, k=2, d=256, f=256, T=96, fmt="int4",
+                       swiglu=True, logits="normal", adapter=True, train=True, seed=2001)
+RAGGED_MX = MoEConfig("ragged_mxfp4", E=5, k=3, d=128, f=192, T=37, fmt="mxfp4", swiglu=True,
+                      logits="normal", adapter=True, train=True, seed=2002, chunk_size=2)
+
+
+def _to(wl, dev):
+    out = {}
+    for key, v in wl.items():
+        if isinstance(v, torch.Tensor):
+            out[key] = v.to(dev)
+        elif isinstance(v, synth.QWeightT):
+            out[key] = v.to(dev)
+        else:
+            out[key] = v
+    return out
+
+
+def _gpu_workload(cfg, T=None):
+    return _to(synth.make_workload(cfg, "cpu", T=T), DEV)
+
+
+# ----------------------------------------------------------------------------- dequant
+
+def test_dequant_int4_exhaustive_bit_exact():
+    # every code x every BF16 scale bit pattern (65536 rows, 64 elements each)
+    R, K = 65536, 64
+    codes = np.tile(np.arange(16, dtype=np.uint8), K // 16)
+    row = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    packed = np.tile(row, (R, 1))
+    scales = np.tile(np.arange(R, dtype=np.uint16), (K // 32, 1))          # [K/32, R]
+    got = moeq.moe_test_dequant(torch.from_numpy(packed).to(DEV),
+                                torch.from_numpy(scales.view(np.int16)).to(DEV).view(torch.bfloat16),
+                                "int4")
+    want = O.dequant_int4_rows(packed, scales.T)
+    g = bf16_bits(got)
+    w = O.bf16_bits_from_values(want)
+    nan_both = np.isnan(want) & np.isnan(f64(got))
+    assert np.array_equal(g[~nan_both], w[~nan_both])
+    assert np.array_equal(np.isnan(want), np.isnan(f64(got)))
+
+
+def test_dequant_mxfp4_exhaustive_bit_exact():
+    R, K = 256, 64
+    codes = np.tile(np.arange(16, dtype=np.uint8), K // 16)
+    row = (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+    packed = np.tile(row, (R, 1))
+    scales = np.tile(np.arange(R, dtype=np.uint8), (K // 32, 1))
+    got = moeq.moe_test_dequant(torch.from_numpy(packed).to(DEV), torch.from_numpy(scales).to(DEV),
+                                "mxfp4")
+    want = O.dequant_mxfp4_rows(packed, scales.T)
+    gv = f64(got)
+    nan_both = np.isnan(want) & np.isnan(gv)
+    assert np.array_equal(np.isnan(want), np.isnan(gv))
+    assert np.array_equal(bf16_bits(got)[~nan_both], O.bf16_bits_from_values(want)[~nan_both])
+
+
+# ----------------------------------------------------------------------------- routing
+
+def _check_routing(r: moeq.Routing, logits, x, k, C, E):
+    topk, gates = O.route_topk(logits.cpu().numpy(), k)
+    g = O.group_by_expert(topk, E, C)
+    assert np.array_equal(r.topk_idx.cpu().numpy(), topk)
+    assert np.allclose(r.gates.cpu().numpy(), gates, rtol=2e-6, atol=1e-7)
+    assert np.array_equal(r.expert_offsets.cpu().numpy(), g.offsets)
+    A = int(r.num_active.item())
+    assert A == g.num_active
+    assert np.array_equal(r.active.cpu().numpy()[:A], g.active)
+    nch = int(r.num_chunks.item())
+    assert nch == g.num_chunks
+    assert np.array_equal(r.chunk_offsets.cpu().numpy()[:nch + 1], g.chunk_offsets)
+    assert np.array_equal(r.perm_token.cpu().numpy(), g.perm_token)
+    assert np.array_equal(r.inv_perm.cpu().numpy(), g.inv_perm)
+    if x is not None:
+        xp = r.x_perm.cpu().view(torch.int16).numpy()
+        assert np.array_equal(xp, x.cpu().view(torch.int16).numpy()[g.perm_token])
+    return g
+
+
+@pytest.mark.parametrize("T,E,k,C", [(1, 4, 4, 1), (37, 5, 3, 2), (64, 8, 2, 8), (1000, 64, 4, 16),
+                                     (130, 384, 8, 32), (4097, 256, 8, 8)])
+def test_route_permute_bit_exact(T, E, k, C):
+    g = torch.Generator().manual_seed(T * 7 + E)
+    logits = torch.randn((T, E), generator=g)
+    logits[: T // 3] = torch.round(logits[: T // 3] * 2) / 2          # many exact ties
+    x = torch.randn((T, 64), generator=g).to(torch.bfloat16)
+    r = moeq.moe_route_permute(logits.to(DEV), x.to(DEV), k, C)
+    torch.cuda.synchronize()
+    _check_routing(r, logits, x, k, C, E)
+
+
+def test_route_uniform_logits_full_size():
+    wl = _gpu_workload(MXFP4_UP)
+    r = moeq.moe_route_permute(wl["logits"], wl["x"], MXFP4_UP.k, MXFP4_UP.chunk_size)
+    torch.cuda.synchronize()
+    _check_routing(r, wl["logits"], wl["x"], MXFP4_UP.k, MXFP4_UP.chunk_size, MXFP4_UP.E)
+
+
+# ----------------------------------------------------------------------------- GEMMs
+
+def _zero_sign_free(bits):
+    # The sum of one exact term and zero products is exact, except that the
+    # sign of a zero weight is lost (-0 + +0 = +0): compare zeros as equal.
+    b = np.array(bits, dtype=np.uint16)
+    b[b == 0x8000] = 0
+    return b
+
+
+def test_one_hot_probe_reads_weights_bit_exact():
+    # a = e_k rows make out[:, n] = W[n, k] exactly: checks layout and placement
+    # of the dequantized tile inside the real GEMM without writing it to memory.
+    for fmt in ("int4", "mxfp4"):
+        gen = torch.Generator().manual_seed(5)
+        E, N, K = 3, 256, 192
+        w = synth.random_qweight(gen, E, N, K, fmt, "cpu", std=0.5)
+        kk = np.array([0, 1, 31, 32, 63, 64, 100, 191])
+        rows_per_e = len(kk)
+        M = E * rows_per_e
+        a = torch.zeros((M, K), dtype=torch.bfloat16)
+        logits = torch.full((M, E), -10.0)
+        for e in range(E):
+            for i, c in enumerate(kk):
+                a[e * rows_per_e + i, c] = 1.0
+                logits[e * rows_per_e + i, e] = 10.0
+        r = moeq.moe_route_permute(logits.to(DEV), a.to(DEV), 1, 2)
+        out = moeq.moe_grouped_qgemm_fwd(r.x_perm, w.to(DEV), r, moeq.EPI_NONE)
+        ow = oracle_qweight(w)
+        got = _zero_sign_free(bf16_bits(out))
+        for e in range(E):
+            W = O.dequant_expert(ow, e)
+            for i, c in enumerate(kk):
+                want = _zero_sign_free(O.bf16_bits_from_values(W[:, c]))
+                assert np.array_equal(got[e * rows_per_e + i], want), (fmt, e, c)
+        # backward orientation: d = e_n rows pick row n of W
+        d = torch.zeros((M, N), dtype=torch.bfloat16)
+        nn = np.array([0, 5, 63, 64, 200, 255, 128, 7])
+        for e in range(E):
+            for i, n in enumerate(nn):
+                d[e * rows_per_e + i, n] = 1.0
+        din = moeq.moe_grouped_qgemm_bwd_dx(d.to(DEV), w.to(DEV), r, moeq.EPI_NONE)
+        got = _zero_sign_free(bf16_bits(din))
+        for e in range(E):
+            W = O.dequant_expert(ow, e)
+            for i, n in enumerate(nn):
+                want = _zero_sign_free(O.bf16_bits_from_values(W[n, :]))
+                assert np.array_equal(got[e * rows_per_e + i], want), (fmt, e, n)
+
+
+def _oracle_weights(wl):
+    out = {}
+    for key in ("w_gu", "w_d", "w_up"):
+        if key in wl:
+            out[key] = oracle_qweight(wl[key])
+    return out
+
+
+def _run_layer_and_compare(cfg, T=None):
+    wl = _gpu_workload(cfg, T)
+    ow = _oracle_weights(wl)
+    R = f64(wl["adapter"]) if cfg.adapter else None
+    st = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], cfg.k, cfg.chunk_size,
+                       adapter=wl.get("adapter"), train=cfg.train)
+    torch.cuda.synchronize()
+    ref = O.moe_forward(f64(wl["x"]), wl["logits"].cpu().numpy(), cfg.k, cfg.chunk_size,
+                        ow["w_gu"], ow["w_d"], R=R)
+    _check_routing(st["routing"], wl["logits"], wl["x"], cfg.k, cfg.chunk_size, cfg.E)
+    assert_close_intermediate(f64(st["h"]), ref["h"], "h")
+    assert_close_intermediate(f64(st["y_perm"]), ref["y_perm"], "y_perm")
+    assert_close_final(f64(st["y"]), ref["y"], "y")
+    if cfg.train:
+        assert_close_intermediate(f64(st["saved_gu"]), ref["saved_gu"], "saved_gu")
+        bw = layer.backward(st, wl["dy"], wl["w_gu"], wl["w_d"], adapter=wl.get("adapter"))
+        torch.cuda.synchronize()
+        rb = O.moe_backward(ref, f64(wl["dy"]), ow["w_gu"], ow["w_d"], R=R)
+        assert np.array_equal(bf16_bits(bw["dy_perm"]), O.bf16_bits_from_values(rb["dy_perm"]))
+        assert_close_intermediate(f64(bw["dgu"]), rb["dgu"], "dgu")
+        assert_close_final(f64(bw["dx"]), rb["dx"], "dx")
+        if cfg.adapter:
+            assert_close_final(bw["d_adapter"].cpu().numpy().astype(np.float64), rb["d_adapter"],
+                               "d_adapter")
+    return st
+
+
+def test_tiny_int4_layer_forward():
+    _run_layer_and_compare(TINY_INT4)
+
+
+def test_tiny_train_forward_backward_with_adapter():
+    _run_layer_and_compare(TINY_TRAIN)
+
+
+def test_ragged_mxfp4_train_with_adapter():
+    _run_layer_and_compare(RAGGED_MX)
+
+
+def test_single_token():
+    _run_layer_and_compare(RAGGED_MX.with_(T=1, seed=2003))
+
+
+def test_adapter_identity_is_bitwise_noop():
+    wl = _gpu_workload(TINY_INT4)
+    eye = torch.eye(32, dtype=torch.bfloat16, device=DEV).expand(TINY_INT4.E, TINY_INT4.d // 32, 32, 32).contiguous()
+    a = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], 2, 8)
+    b = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], 2, 8, adapter=eye)
+    assert torch.equal(a["y"], b["y"])
+
+
+def test_outputs_identical_across_chunk_sizes():
+    cfg = TINY_TRAIN
+    wl = _gpu_workload(cfg)
+    ys = []
+    for C in (1, 3, 8, 16, 32):
+        st = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], cfg.k, C,
+                           adapter=wl["adapter"], train=True)
+        bw = layer.backward(st, wl["dy"], wl["w_gu"], wl["w_d"], adapter=wl["adapter"])
+        ys.append((st["y"].clone(), bw["dx"].clone(), bw["d_adapter"].clone()))
+    for y, dx, da in ys[1:]:
+        assert torch.equal(y, ys[0][0]) and torch.equal(dx, ys[0][1]) and torch.equal(da, ys[0][2])
+
+
+def test_mxfp4_up_projection_full_size():
+    """The bench workload at its full size: every output compared with the oracle."""
+    cfg = MXFP4_UP
+    wl = _gpu_workload(cfg)
+    st = layer.up_projection(wl["x"], wl["logits"], wl["w_up"], cfg.k, cfg.chunk_size)
+    torch.cuda.synchronize()
+    ref = O.up_projection(f64(wl["x"]), wl["logits"].cpu().numpy(), cfg.k, cfg.chunk_size,
+                          oracle_qweight(wl["w_up"]))
+    _check_routing(st["routing"], wl["logits"], wl["x"], cfg.k, cfg.chunk_size, cfg.E)
+    assert_close_final(f64(st["out"]), ref["out"], "out")
+
+
+def test_device_error_word_is_clear_after_runs():
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
