@@ -1,0 +1,562 @@
+"""Throughput of the low-bit MoE hot path on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole path over one batch of synthetic tokens. The
+default workload is the single grouped MXFP4 up-projection (E=64, top-4,
+d=2048, f=1024, T=1024 tokens per GPU): route -> permute -> fused dequant +
+grouped GEMM. Other workloads (--workload) run the SwiGLU layer forward, or
+forward + backward with the adapter.
+
+Timing: inputs live in HBM; four independent input sets (weights, tokens,
+logits, outputs; together larger than the 126 MB L2) are used in rotation so
+no step finds its data in L2. Each step is one CUDA-graph replay; the K timed
+steps are bracketed by a barrier and a device synchronize on both sides and
+timed with CUDA events on the launching stream; the max over ranks is
+reported. With N > 1 GPUs every rank runs its own token batch against the
+same (replicated) weights: weak scaling, no collective on the data path.
+
+--impl reference times the CPU oracle (plain float64 numpy) on this machine's host
+cores, rank 0 only, on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "grouped low-bit MoE GEMM TFLOP/s and weight GB/s (fraction of roofline)"
+ROTATE = 4
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="mxfp4_up")
+    ap.add_argument("--chunk", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def _workloads():
+    from quantized_rl_fine_b200 import configs as C
+    w = {
+        "mxfp4_up": C.MXFP4_UP,
+        "tiny_int4": C.TINY_INT4,
+        "zipf_mxfp4": C.ZIPF_MXFP4,
+        "train_int4": C.TRAIN_INT4,
+    }
+    for T in C.TRILLION_T_SWEEP:
+        w[f"trillion_int4_T{T}"] = C.TRILLION_INT4.with_(T=T)
+    return w
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def _accounting(cfg, counts):
+    """Useful flops and algorithmic bytes of one step from the per-expert row counts."""
+    from quantized_rl_fine_b200 import accounting as A
+    M = int(sum(counts))
+    act = [c for c in counts if c > 0]
+    d, f = cfg.d, cfg.f
+    if not cfg.swiglu:
+        flops = A.gemm_flops(counts, f, d)
+        wbytes = A.active_weight_bytes(counts, f, d, cfg.fmt)
+        gemm = dict(flops=flops, bytes=wbytes + M * d * 2 + M * f * 2, wbytes=wbytes)
+        return dict(flops=flops, wbytes=wbytes, gemm=gemm)
+    gu_flops = A.gemm_flops(counts, 2 * f, d)
+    dn_flops = A.gemm_flops(counts, d, f)
+    gu_w = A.active_weight_bytes(counts, 2 * f, d, cfg.fmt)
+    dn_w = A.active_weight_bytes(counts, d, f, cfg.fmt)
+    flops = gu_flops + dn_flops + (2 * M * d * 32 if cfg.adapter else 0)
+    wbytes = gu_w + dn_w
+    if cfg.train:
+        flops += gu_flops + dn_flops + (4 * M * d * 32 if cfg.adapter else 0)
+        wbytes *= 2
+    gemm = dict(flops=gu_flops, bytes=gu_w + M * d * 2 + M * f * 2 + (M * 2 * f * 2 if cfg.train else 0),
+                wbytes=gu_w)
+    return dict(flops=flops, wbytes=wbytes, gemm=gemm)
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {
+        0x0000000000000004: "sw_power_cap", 0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown", 0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown", 0x0000000000000002: "applications_clocks_setting",
+    }
+
+    def __init__(self, cuda_index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._nv = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(cuda_index)
+            want = (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                pci = pynvml.nvmlDeviceGetPciInfo(h)
+                if (pci.domain, pci.bus, pci.device) == want:
+                    self._h = h
+                    self._nv = pynvml
+                    break
+            if self._nv is not None:
+                self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                mask = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- profiles
+
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_rl_fine_b200", "csrc")
+    for name in ("gemm.cu", "dequant.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(workload):
+    """DRAM bytes per launch of the grouped GEMM from the committed ncu summary,
+    when it was taken on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"grouped_qgemm_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", text)
+    m_bytes = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != _kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm=p["hbm_gbs"], tensor=p["bf16_tflops"], tensor_sust=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sust=1400.0, source="fallback")
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def _slice_features(w, e, nf):
+    """Expert e of an oracle weight stack, restricted to its first nf rows."""
+    import oracle as O
+    return O.QWeight(w.fmt, w.packed[e:e + 1, :nf], w.scales[e:e + 1, :, :nf])
+
+
+def _oracle_step_sample(cfg, wl_np, n_experts, frac=1.0):
+    """One oracle step restricted to the rows of the first n_experts active
+    experts; with frac < 1 (one expert), to the first frac of its output
+    features as well. Returns (seconds, useful flops of the sample)."""
+    import numpy as np
+    import oracle as O
+    t0 = time.perf_counter()
+    topk, gates = O.route_topk(wl_np["logits"], cfg.k)
+    g = O.group_by_expert(topk, cfg.E, cfg.chunk_size)
+    flops = 0
+    for e in g.active[:n_experts]:
+        rows = np.arange(g.offsets[e], g.offsets[e + 1])
+        xp = wl_np["x"][g.perm_token[rows]]
+        re_ = np.zeros(len(rows), dtype=np.int64)
+        if not cfg.swiglu:
+            nf = max(64, int(cfg.f * frac) // 64 * 64)
+            O.grouped_gemm_fwd(xp, re_, _slice_features(wl_np["w_up"], e, nf))
+            flops += 2 * len(rows) * nf * cfg.d
+            continue
+        nf = max(64, int(cfg.f * frac) // 64 * 64)        # H features of the sample
+        wgu = wl_np["w_gu"]
+        gate_up = O.QWeight(wgu.fmt, np.concatenate([wgu.packed[e:e + 1, :nf],
+                                                     wgu.packed[e:e + 1, cfg.f:cfg.f + nf]], 1),
+                            np.concatenate([wgu.scales[e:e + 1, :, :nf],
+                                            wgu.scales[e:e + 1, :, cfg.f:cfg.f + nf]], 2))
+        wd = wl_np["w_d"]
+        down = O.QWeight(wd.fmt, wd.packed[e:e + 1, :, :nf // 2], wd.scales[e:e + 1, :nf // 32, :])
+        xa = O.adapter_fwd(xp, re_, wl_np["R"][e:e + 1]) if cfg.adapter else xp
+        h, saved = O.grouped_gemm_fwd(xa, re_, gate_up, O.EPI_SWIGLU)
+        O.grouped_gemm_fwd(h, re_, down)
+        step = 2 * len(rows) * (2 * nf * cfg.d + nf * cfg.d)
+        if cfg.train:
+            dyp = wl_np["dy"][g.perm_token[rows]]
+            dgu = O.grouped_gemm_bwd_dx(dyp, re_, down, O.EPI_SWIGLU_BWD, saved)
+            dxa = O.grouped_gemm_bwd_dx(dgu, re_, gate_up)
+            if cfg.adapter:
+                O.adapter_bwd(xp, dxa, re_, wl_np["R"][e:e + 1], 1)
+            step *= 2
+        flops += step
+    return time.perf_counter() - t0, flops
+
+
+def _sample_size(cfg, wl, budget_s):
+    """(n_experts, frac) whose oracle step takes about budget_s seconds."""
+    import oracle as O
+    t_one, _ = _oracle_step_sample(cfg, wl, 1)
+    topk, _ = O.route_topk(wl["logits"], cfg.k)
+    A = O.group_by_expert(topk, cfg.E, cfg.chunk_size).num_active
+    if t_one <= budget_s:
+        return int(max(1, min(A, budget_s / max(t_one, 1e-4)))), 1.0, A
+    return 1, max(64.0 / cfg.f, budget_s / t_one), A
+
+
+def _numpy_workload(cfg, T):
+    import numpy as np
+    import torch
+    import oracle as O
+    from quantized_rl_fine_b200 import synth
+    wl = synth.make_workload(cfg, "cpu", T=T)
+
+    def qw(w):
+        sc = w.scales.view(torch.int16).numpy().view(np.uint16) if w.fmt == "int4" else w.scales.numpy()
+        return O.QWeight(w.fmt, w.packed.numpy(), sc)
+    out = {"logits": wl["logits"].numpy(), "x": wl["x"].float().numpy().astype(np.float64)}
+    for key in ("w_up", "w_gu", "w_d"):
+        if key in wl:
+            out[key] = qw(wl[key])
+    if cfg.adapter:
+        out["R"] = wl["adapter"].float().numpy().astype(np.float64)
+    if cfg.train:
+        out["dy"] = wl["dy"].float().numpy().astype(np.float64)
+    return out
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        return os.cpu_count()
+
+
+def _cpu_baseline(cfg, budget_s=20.0):
+    """Oracle throughput on a bounded sample (about budget_s seconds), timed once."""
+    wl = _numpy_workload(cfg, cfg.T)
+    n, frac, A = _sample_size(cfg, wl, budget_s)
+    secs, flops = _oracle_step_sample(cfg, wl, n, frac)
+    part = "all of their output features" if frac >= 1.0 else f"{frac:.3f} of its output features"
+    return dict(value=flops / secs / 1e12, unit="TFLOP/s", cores=_blas_threads(), kind="oracle",
+                sample=f"routing of all {cfg.T} tokens + the rows of {n} of {A} active experts, "
+                       f"{part}; one pass of the float64 numpy oracle, "
+                       f"{flops / 1e9:.2f} GFLOP in {secs:.2f} s")
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = _numpy_workload(cfg, cfg.T)
+    per_step = 150.0 / max(1, args.steps + args.warmup)
+    n, frac, A = _sample_size(cfg, wl, per_step)
+    for _ in range(args.warmup):
+        _oracle_step_sample(cfg, wl, n, frac)
+    secs = flops = 0.0
+    for _ in range(args.steps):
+        s, fl = _oracle_step_sample(cfg, wl, n, frac)
+        secs += s
+        flops += fl
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "E": cfg.E, "k": cfg.k, "d": cfg.d, "f": cfg.f,
+                   "T": cfg.T, "fmt": cfg.fmt},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: routing of all {cfg.T} tokens + the GEMMs of "
+                                   f"the rows of {n} of {A} active experts"
+                                   + ("" if frac >= 1.0 else f", {frac:.3f} of the output features")},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def _make_sets(cfg, device, rank):
+    from quantized_rl_fine_b200 import synth
+    sets = []
+    for i in range(ROTATE):
+        c = cfg.with_(seed=cfg.seed + 7919 * i + 104729 * rank)
+        wl = synth.make_workload(c, device)
+        sets.append(wl)
+    return sets
+
+
+def _step_fn(cfg, chunk):
+    from quantized_rl_fine_b200 import layer
+
+    def step(wl):
+        if not cfg.swiglu:
+            return layer.up_projection(wl["x"], wl["logits"], wl["w_up"], cfg.k, chunk)
+        st = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], cfg.k, chunk,
+                           adapter=wl.get("adapter"), train=cfg.train)
+        if cfg.train:
+            bw = layer.backward(st, wl["dy"], wl["w_gu"], wl["w_d"], adapter=wl.get("adapter"))
+            st.update(bw)
+        return st
+    return step
+
+
+def _launches_per_step(cfg):
+    route = 3
+    if not cfg.swiglu:
+        return route + 1
+    n = route + 2 + 1                           # gate/up, down, combine
+    if cfg.adapter:
+        n += 1                                  # adapter apply
+    if cfg.train:
+        n += 1 + 2 + 1                          # scatter, two bwd GEMMs, unpermute-sum
+        if cfg.adapter:
+            n += 2                              # adapter backward (dx, dR)
+    return n
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    from quantized_rl_fine_b200 import moeq
+    from quantized_rl_fine_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    moeq.lib()
+
+    chunk = args.chunk or cfg.chunk_size
+    step = _step_fn(cfg, chunk)
+    sets = _make_sets(cfg, dev, rank)
+    torch.cuda.synchronize()
+
+    # routing statistics of set 0 (outside any timed region)
+    r0 = moeq.moe_route_permute(sets[0]["logits"], None, cfg.k, chunk)
+    counts = (r0.expert_offsets[1:] - r0.expert_offsets[:-1]).cpu().tolist()
+    acc = _accounting(cfg, counts)
+
+    # eager warm-up (sets attributes, builds maps), then one graph per input set
+    for wl in sets:
+        step(wl)
+    torch.cuda.synchronize()
+    graphs, keep = [], []
+    for wl in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            keep.append(step(wl))
+        graphs.append(g)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------------- timed region
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            graphs[i % ROTATE].replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / args.steps
+    assert moeq.moe_get_device_error() == 0
+
+    # ---------------------------------------------------------------- dominant kernel alone
+    from quantized_rl_fine_b200 import layer
+    gemm_graphs = []
+    for i, wl in enumerate(sets):
+        st = keep[i]
+        r = st["routing"]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if not cfg.swiglu:
+                moeq.moe_grouped_qgemm_fwd(r.x_perm, wl["w_up"], r, moeq.EPI_NONE)
+            else:
+                moeq.moe_grouped_qgemm_fwd(r.x_perm, wl["w_gu"], r, moeq.EPI_SWIGLU,
+                                           adapter=wl.get("adapter"), save_gu=cfg.train)
+        gemm_graphs.append(g)
+    for i in range(max(3, args.warmup)):
+        gemm_graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_k = max(args.steps, 20)
+    ka.record(stream)
+    for i in range(n_k):
+        gemm_graphs[i % ROTATE].replay()
+    kb.record(stream)
+    torch.cuda.synchronize()
+    k_ms = ka.elapsed_time(kb) / n_k
+
+    # ---------------------------------------------------------------- end to end via host buffers
+    host = []
+    for wl in sets:
+        hx = wl["x"].cpu().pin_memory()
+        hl = wl["logits"].cpu().pin_memory()
+        hy = wl["dy"].cpu().pin_memory() if cfg.train else None
+        host.append((hx, hl, hy))
+    out_key = "out" if not cfg.swiglu else ("dx" if cfg.train else "y")
+    out_shape = keep[0][out_key].shape
+    hout = [torch.empty(out_shape, dtype=torch.bfloat16).pin_memory() for _ in range(ROTATE)]
+    h2d = sum(t.numel() * t.element_size() for t in host[0] if t is not None)
+    d2h = hout[0].numel() * hout[0].element_size()
+
+    def e2e_step(i):
+        hx, hl, hy = host[i % ROTATE]
+        wl = sets[i % ROTATE]
+        wl["x"].copy_(hx, non_blocking=True)
+        wl["logits"].copy_(hl, non_blocking=True)
+        if hy is not None:
+            wl["dy"].copy_(hy, non_blocking=True)
+        graphs[i % ROTATE].replay()
+        hout[i % ROTATE].copy_(keep[i % ROTATE][out_key], non_blocking=True)
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    assert moeq.moe_get_device_error() == 0
+
+    # ---------------------------------------------------------------- report
+    del graphs, gemm_graphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks = _peaks()
+    step_flops = acc["flops"]
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    gemm = acc["gemm"]
+    k_bytes_rate = gemm["bytes"] / (k_ms * 1e-3) / 1e9
+    k_flop_rate = gemm["flops"] / (k_ms * 1e-3) / 1e12
+    t_hbm = gemm["bytes"] / (peaks["hbm"] * 1e9)
+    t_tc = gemm["flops"] / (peaks["tensor"] * 1e12)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": k_bytes_rate, "peak": peaks["hbm"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": k_flop_rate, "peak": peaks["tensor"], "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = _profiled_traffic(args.workload)
+    roof["kernel"] = "grouped_qgemm_kernel (fwd" + (", SwiGLU" if cfg.swiglu else "") + ")"
+    roof["kernel_ms"] = k_ms
+    roof["algorithmic_bytes"] = gemm["bytes"]
+    roof["algorithmic_flops"] = gemm["flops"]
+    roof["peak_source"] = peaks["source"] + " (burst)"
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "E": cfg.E, "k": cfg.k, "d": cfg.d, "f": cfg.f,
+                   "T_per_gpu": cfg.T, "fmt": cfg.fmt, "chunk_size": chunk,
+                   "adapter": cfg.adapter, "train": cfg.train,
+                   "l2": f"{ROTATE} rotating input sets, larger than L2 together",
+                   "parallelism": f"dp{world} (replicated weights, own tokens per GPU)"},
+        "weight_gbs": world * acc["wbytes"] / (ms_per_step * 1e-3) / 1e9,
+        "roofline": roof,
+        "e2e": {"value": world * step_flops / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e_ms / args.steps},
+        "gpu_launches": _launches_per_step(cfg) * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = _cpu_baseline(cfg)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _args()
+    cfg = _workloads()[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

@@ -35,9 +35,11 @@
  *    of its time budget, an offsets table inconsistent with M) sets a device
  *    error word that moe_get_device_error reads and clears.
  *  - Workspace: calls that take (ws, ws_bytes) report the bytes they need
- *    when ws == NULL (then nothing is launched and *ws_bytes is written);
- *    otherwise *ws_bytes must hold the size of ws, which must be at least the
- *    queried size and 256-byte aligned.
+ *    when ws == NULL and ws_bytes != NULL (then nothing is launched and
+ *    *ws_bytes is written). With ws == NULL and ws_bytes == NULL the call
+ *    runs without a workspace, which is valid only when the query returned
+ *    0. Otherwise *ws_bytes must hold the size of ws, which must be at least
+ *    the queried size and 256-byte aligned.
  *  - BF16 tensors are row-major with the last dimension contiguous.
  *
  * Weight formats (moe_qweight)
@@ -159,7 +161,7 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
  *           MOE_EPI_SWIGLU: out [M][N/2] = bf16(silu(acc[:, :N/2]) *
  *           acc[:, N/2:]) and, if saved_gu != NULL, saved_gu [M][N] =
  *           bf16(acc) (kept for the backward).
- *  ws       scratch: the tile schedule, plus M*K bf16 for a' with an adapter.
+ *  ws       scratch: M*K bf16 for a' with an adapter; none without one.
  * Experts with no rows cost nothing: their weight bytes are never read.
  */
 moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
@@ -184,7 +186,7 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
  *             s = sigmoid(g): din [M][2K] = bf16([dh*u*s*(1+g*(1-s)) |
  *             dh*g*s]). adapter must be NULL.
  *  adapter, a, d_adapter: NULL, or all three given (a = the forward's a).
- *  ws       scratch: the tile schedule, plus M*K bf16 for dx' with an adapter.
+ *  ws       scratch: M*K bf16 for dx' with an adapter; none without one.
  */
 moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweight* w,
                                     const moe_groups* g, int32_t epi, const void* saved_gu,

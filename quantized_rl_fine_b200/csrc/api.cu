@@ -133,7 +133,6 @@ struct GemmPlan {
   int BN, stages, grid, n_ftiles;
   uint32_t stage_bytes;
   size_t smem;
-  size_t sched_bytes;
 };
 
 // F: output features; tile_f: output features per tile (128, or 64 for the
@@ -144,24 +143,41 @@ GemmPlan plan_gemm(int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) 
   pl.stage_bytes = gemm_stage_bytes(pl.BN, fmt);
   const int avail = max_smem_optin();
   int stages = 8;
-  while (stages > 2 && static_cast<int>(stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages)) > avail)
+  while (stages > 2 &&
+         static_cast<int>(stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, w->E)) > avail)
     --stages;
   pl.stages = stages;
-  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages);
+  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, w->E);
   pl.n_ftiles = (F + tile_f - 1) / tile_f;
   const int64_t bound = static_cast<int64_t>(pl.n_ftiles) *
                         (std::min<int64_t>(w->E, M) + (M + pl.BN - 1) / pl.BN);
   pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound)));
-  pl.sched_bytes = align_up(static_cast<size_t>(w->E + 3) * sizeof(int32_t), 256);
   return pl;
 }
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Runs one grouped GEMM launch (schedule + main kernel) on `a_or_dout` rows.
+// Workspace convention: ws == NULL with ws_bytes != NULL is a size query
+// (writes *ws_bytes). ws == NULL with ws_bytes == NULL runs without a
+// workspace, which is valid only when the call needs none. Otherwise
+// *ws_bytes must cover `need` and ws must be 256-byte aligned.
+moe_status check_workspace(void* ws, size_t* ws_bytes, size_t need) {
+  if (!ws) {
+    if (ws_bytes) {
+      *ws_bytes = need;
+      return MOE_OK;
+    }
+    return need == 0 ? MOE_OK : MOE_ERR_WORKSPACE;
+  }
+  if (!ws_bytes || *ws_bytes < need) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  return MOE_OK;
+}
+
+// Runs one grouped GEMM launch over the rows of `bmat` (a, a' or dout).
 moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qweight* w,
-                    const moe_groups* g, void* out, int64_t ldo, void* saved, int32_t* sched,
-                    const GemmPlan& pl, cudaStream_t s) {
+                    const moe_groups* g, void* out, int64_t ldo, void* saved, const GemmPlan& pl,
+                    cudaStream_t s) {
   const int F = (mode == kModeFwd) ? (epi == MOE_EPI_SWIGLU ? w->N / 2 : w->N) : w->K;
   const int R = (mode == kModeFwd) ? w->K : w->N;
   CUtensorMap tb, tw, ts;
@@ -188,18 +204,16 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
                      CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
   }
-  cudaError_t e = launch_build_schedule(g->expert_offsets, g->active, g->num_active, sched, w->E,
-                                        static_cast<int>(M), pl.BN, pl.n_ftiles, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
   GemmArgs p;
   p.offsets = g->expert_offsets;
   p.active = g->active;
-  p.sched = sched;
+  p.num_active = g->num_active;
   p.E = w->E;
   p.N = w->N;
   p.K = w->K;
   p.M = static_cast<int32_t>(M);
   p.BN = pl.BN;
+  p.n_ftiles = pl.n_ftiles;
   p.acc_cols = (pl.BN + 31) / 32 * 32;
   p.tmem_cols = next_pow2(2 * p.acc_cols);
   p.F = F;
@@ -240,18 +254,14 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
                              int32_t* chunk_offsets, int32_t* num_chunks, int32_t* perm_token,
                              int32_t* inv_perm, void* x_perm, void* ws, size_t* ws_bytes,
                              void* stream) {
-  if (!ws_bytes) return MOE_ERR_INVALID_ARG;
   if (T < 1 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || chunk_size < 1)
     return MOE_ERR_INVALID_ARG;
   if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   const int nblk = route_num_blocks(T);
   const size_t need = align_up(static_cast<size_t>(nblk) * E * sizeof(int32_t), 256);
-  if (!ws) {
-    *ws_bytes = need;
-    return MOE_OK;
-  }
-  if (*ws_bytes < need) return MOE_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  moe_status st = check_workspace(ws, ws_bytes, need);
+  if (st != MOE_OK) return st;
+  if (!ws) return MOE_OK;   // size query
   const void* ptrs[] = {logits, topk_idx, gates, expert_offsets, active, num_active,
                         chunk_offsets, num_chunks, perm_token, inv_perm};
   for (const void* p : ptrs) {
@@ -271,7 +281,6 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
 moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
                                  const moe_groups* g, const void* adapter, int32_t epi, void* out,
                                  void* saved_gu, void* ws, size_t* ws_bytes, void* stream) {
-  if (!ws_bytes) return MOE_ERR_INVALID_ARG;
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -279,14 +288,9 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
   if (epi == MOE_EPI_SWIGLU && w->N % 128 != 0) return MOE_ERR_UNSUPPORTED;
   const int F = (epi == MOE_EPI_SWIGLU) ? w->N / 2 : w->N;
   const GemmPlan pl = plan_gemm(M, w, F, epi == MOE_EPI_SWIGLU ? 64 : 128, w->fmt);
-  const size_t xa_bytes = adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
-  const size_t need = pl.sched_bytes + xa_bytes;
-  if (!ws) {
-    *ws_bytes = need;
-    return MOE_OK;
-  }
-  if (*ws_bytes < need) return MOE_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  const size_t need = adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
+  if ((st = check_workspace(ws, ws_bytes, need)) != MOE_OK) return st;
+  if (!ws && ws_bytes) return MOE_OK;   // size query
   if ((st = check_groups(g, w->E)) != MOE_OK) return st;
   if (!a || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(out) || (saved_gu && !aligned16(saved_gu)) ||
@@ -294,23 +298,21 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
     return MOE_ERR_MISALIGNED;
   if (saved_gu && epi != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t* sched = static_cast<int32_t*>(ws);
   const void* bmat = a;
   if (adapter) {
-    void* xa = static_cast<uint8_t*>(ws) + pl.sched_bytes;
+    void* xa = ws;
     cudaError_t e = launch_adapter_apply(a, adapter, g->expert_offsets, w->E, static_cast<int>(M),
                                          w->K, xa, false, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     bmat = xa;
   }
-  return run_gemm(kModeFwd, epi, bmat, M, w, g, out, F, saved_gu, sched, pl, s);
+  return run_gemm(kModeFwd, epi, bmat, M, w, g, out, F, saved_gu, pl, s);
 }
 
 moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweight* w,
                                     const moe_groups* g, int32_t epi, const void* saved_gu,
                                     const void* adapter, const void* a, void* din,
                                     float* d_adapter, void* ws, size_t* ws_bytes, void* stream) {
-  if (!ws_bytes) return MOE_ERR_INVALID_ARG;
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -320,14 +322,9 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
   if (!with_adapter && (a || d_adapter)) return MOE_ERR_INVALID_ARG;
   if (epi == MOE_EPI_SWIGLU_BWD && !saved_gu) return MOE_ERR_INVALID_ARG;
   const GemmPlan pl = plan_gemm(M, w, w->K, 128, w->fmt);
-  const size_t dx_bytes = with_adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
-  const size_t need = pl.sched_bytes + dx_bytes;
-  if (!ws) {
-    *ws_bytes = need;
-    return MOE_OK;
-  }
-  if (*ws_bytes < need) return MOE_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_MISALIGNED;
+  const size_t need = with_adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
+  if ((st = check_workspace(ws, ws_bytes, need)) != MOE_OK) return st;
+  if (!ws && ws_bytes) return MOE_OK;   // size query
   if ((st = check_groups(g, w->E)) != MOE_OK) return st;
   if (!dout || !din) return MOE_ERR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(din) || (saved_gu && !aligned16(saved_gu)) ||
@@ -335,16 +332,15 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
       (d_adapter && !aligned16(d_adapter)))
     return MOE_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t* sched = static_cast<int32_t*>(ws);
   if (epi == MOE_EPI_SWIGLU_BWD) {
     return run_gemm(kModeBwd, epi, dout, M, w, g, din, 2 * static_cast<int64_t>(w->K),
-                    const_cast<void*>(saved_gu), sched, pl, s);
+                    const_cast<void*>(saved_gu), pl, s);
   }
   if (!with_adapter) {
-    return run_gemm(kModeBwd, epi, dout, M, w, g, din, w->K, nullptr, sched, pl, s);
+    return run_gemm(kModeBwd, epi, dout, M, w, g, din, w->K, nullptr, pl, s);
   }
-  void* dxa = static_cast<uint8_t*>(ws) + pl.sched_bytes;
-  st = run_gemm(kModeBwd, epi, dout, M, w, g, dxa, w->K, nullptr, sched, pl, s);
+  void* dxa = ws;
+  st = run_gemm(kModeBwd, epi, dout, M, w, g, dxa, w->K, nullptr, pl, s);
   if (st != MOE_OK) return st;
   cudaError_t e = launch_adapter_apply(dxa, adapter, g->expert_offsets, w->E, static_cast<int>(M),
                                        w->K, din, true, s);

@@ -83,8 +83,8 @@ struct Tile {
   int e, ft, row0, row_end;
 };
 
-// Tile t of the device tile list: active index a with tile_start[a] <= t,
-// then feature tile major, token tile minor inside the expert.
+// Tile t of the tile list: active index a with tile_start[a] <= t (shared
+// memory), then feature tile major, token tile minor inside the expert.
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* tile_start, int A,
                                             int t) {
   int lo = 0, hi = A - 1;
@@ -102,6 +102,59 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* ti
   r.row0 = seg0 + (local - r.ft * nrt) * p.BN;
   r.row_end = seg1;
   return r;
+}
+
+// Every CTA builds the tile list of the launch in shared memory:
+// tile_start[a] = sum over active experts a' < a of n_ftiles * ceil(m_e / BN),
+// tile_start[A] = total. Offsets that do not describe M rows give an empty
+// list and raise the device error. Returns A (0 when inconsistent).
+__device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* warp_tot) {
+  const int nthr = blockDim.x;
+  const int tid = threadIdx.x;
+  const int A_raw = *p.num_active;
+  const bool bad = (A_raw < 0 || A_raw > p.E || p.offsets[0] != 0 || p.offsets[p.E] != p.M);
+  if (bad) {
+    if (tid == 0) {
+      if (blockIdx.x == 0) raise_device_error(MOE_DEVERR_BAD_OFFSETS);
+      tile_start[0] = 0;
+    }
+    __syncthreads();
+    return 0;
+  }
+  const int A = A_raw;
+  const int per = (A + nthr - 1) / nthr;           // experts per thread (<= 3 for A <= 1024)
+  const int a0 = min(A, tid * per), a1 = min(A, a0 + per);
+  int local = 0;
+  for (int a = a0; a < a1; ++a) {
+    const int e = p.active[a];
+    const int m = p.offsets[e + 1] - p.offsets[e];
+    local += p.n_ftiles * ((m + p.BN - 1) / p.BN);
+  }
+  const int lane = tid & 31, w = tid >> 5, nw = nthr >> 5;
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[w] = x;
+  __syncthreads();
+  int before = 0;
+  for (int i = 0; i < w; ++i) before += warp_tot[i];
+  int run = before + x - local;                     // exclusive prefix of this thread
+  for (int a = a0; a < a1; ++a) {
+    tile_start[a] = run;
+    const int e = p.active[a];
+    const int m = p.offsets[e + 1] - p.offsets[e];
+    run += p.n_ftiles * ((m + p.BN - 1) / p.BN);
+  }
+  if (tid == nthr - 1) {
+    int total = 0;
+    for (int i = 0; i < nw; ++i) total += warp_tot[i];
+    tile_start[A] = total;
+  }
+  __syncthreads();
+  return A;
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
@@ -137,6 +190,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const uint32_t drain_bar = bars + 8u * (3 * S + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (3 * S + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* warp_tot = reinterpret_cast<int32_t*>(tmem_slot + 4);          // [32]
+  int32_t* tile_start = warp_tot + 32;                                      // [E + 1]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -166,9 +221,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int A = p.sched[0];
-  const int total = p.sched[1];
-  const int32_t* tile_start = p.sched + 2;
+  const int A = build_tile_list(p, tile_start, warp_tot);
+  const int total = tile_start[A];
   const int nkb = p.R / kStageK;
   const int N = p.N, K = p.K;
 
@@ -405,68 +459,6 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
 }
 
-// Tile list of one launch, written to sched = {A, total, tile_start[0..A]}:
-// tile_start[a] = sum over active experts a' < a of n_ftiles * ceil(m_e / BN).
-// Inconsistent offsets publish an empty list and raise the device error.
-// One block of 1024 threads (A <= E <= 1024).
-__global__ void build_schedule_kernel(const int32_t* __restrict__ offsets,
-                                      const int32_t* __restrict__ active,
-                                      const int32_t* __restrict__ num_active,
-                                      int32_t* __restrict__ sched, int E, int M, int BN,
-                                      int n_ftiles) {
-  __shared__ int32_t warp_sums[32];
-  const int A = *num_active;
-  const bool bad = (A < 0 || A > E || offsets[0] != 0 || offsets[E] != M);
-  if (bad) {
-    if (threadIdx.x == 0) {
-      raise_device_error(MOE_DEVERR_BAD_OFFSETS);
-      sched[0] = 0;
-      sched[1] = 0;
-      sched[2] = 0;
-    }
-    return;
-  }
-  const int a = threadIdx.x;
-  int v = 0;
-  if (a < A) {
-    const int e = active[a];
-    const int m = offsets[e + 1] - offsets[e];
-    v = n_ftiles * ((m + BN - 1) / BN);
-  }
-  const int lane = a & 31, w = a >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sums[w] = x;
-  __syncthreads();
-  if (w == 0) {
-    int s = warp_sums[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    warp_sums[lane] = s;
-  }
-  __syncthreads();
-  const int incl = x + (w > 0 ? warp_sums[w - 1] : 0);
-  if (a < A) sched[2 + a] = incl - v;
-  if (a == A - 1) {
-    sched[2 + A] = incl;
-    sched[1] = incl;
-  }
-  if (a == 0) {
-    sched[0] = A;
-    if (A == 0) {
-      sched[1] = 0;
-      sched[2] = 0;
-    }
-  }
-}
-
 }  // namespace
 
 template <int MODE, int FMT, int EPI>
@@ -474,9 +466,18 @@ static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorM
                                           const CUtensorMap& ts, const GemmArgs& p, int grid,
                                           size_t smem, cudaStream_t s) {
   auto k = grouped_qgemm_kernel<MODE, FMT, EPI>;
-  cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  // Raise the dynamic shared-memory limit once per (device, kernel); later
+  // calls, including ones under stream capture, skip it.
+  static int set_for[64] = {0};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (set_for[dev] < static_cast<int>(smem)) {
+    err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (err != cudaSuccess) return err;
+    set_for[dev] = 227 * 1024;
+  }
   k<<<grid, kThreads, smem, s>>>(tb, tw, ts, p);
   return cudaGetLastError();
 }
@@ -499,22 +500,15 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& 
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_build_schedule(const int32_t* offsets, const int32_t* active,
-                                  const int32_t* num_active, int32_t* sched, int E, int M,
-                                  int BN, int n_ftiles, cudaStream_t s) {
-  build_schedule_kernel<<<1, 1024, 0, s>>>(offsets, active, num_active, sched, E, M, BN,
-                                           n_ftiles);
-  return cudaGetLastError();
-}
-
 uint32_t gemm_stage_bytes(int BN, int fmt) {
   const uint32_t sc = 256u * (fmt == MOE_W_INT4_G32_BF16 ? 2u : 1u);
   const uint32_t b = kABytes + static_cast<uint32_t>(BN) * 128u + kWqBytes + sc;
   return (b + 1023u) & ~1023u;
 }
 
-uint32_t gemm_fixed_smem_bytes(int stages) {
-  return 8u * (3u * stages + 5u) + 16u + 1024u;   // barriers, TMEM slot, abort flag, alignment
+uint32_t gemm_fixed_smem_bytes(int stages, int E) {
+  // barriers, TMEM slot + abort flag (16 B), warp totals, tile list, alignment slack
+  return 8u * (3u * stages + 5u) + 16u + 32u * 4u + static_cast<uint32_t>(E + 1) * 4u + 1024u;
 }
 
 }  // namespace moeq

@@ -14,10 +14,11 @@ constexpr int kModeBwd = 1;   // D[f, t] = sum_n W[e][n][f] dout[t][n]
 struct GemmArgs {
   const int32_t* offsets;     // [E+1] expert row offsets
   const int32_t* active;      // [E] active experts (ascending)
-  const int32_t* sched;       // [E+3]: {A, total tiles, tile_start[0..A]}
+  const int32_t* num_active;  // [1] number of active experts
   int32_t E, N, K;            // weight stack dims, W[e] is [N][K]
   int32_t M;                  // rows of a / dout / out
   int32_t BN;                 // token rows per tile (multiple of 16, <= 256)
+  int32_t n_ftiles;           // feature tiles per expert
   int32_t acc_cols;           // TMEM columns per accumulator buffer (>= BN, multiple of 32)
   int32_t tmem_cols;          // TMEM columns allocated (power of two, >= 2 * acc_cols)
   int32_t F;                  // output features (fwd: N or N/2 with SwiGLU; bwd: K)
@@ -32,11 +33,8 @@ struct GemmArgs {
 cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& tb,
                                  const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
                                  int grid, size_t smem, cudaStream_t s);
-cudaError_t launch_build_schedule(const int32_t* offsets, const int32_t* active,
-                                  const int32_t* num_active, int32_t* sched, int E, int M, int BN,
-                                  int n_ftiles, cudaStream_t s);
 uint32_t gemm_stage_bytes(int BN, int fmt);
-uint32_t gemm_fixed_smem_bytes(int stages);
+uint32_t gemm_fixed_smem_bytes(int stages, int E);
 constexpr int kGemmThreads = 384;
 
 }  // namespace moeq

@@ -109,8 +109,12 @@ def _require_cuda(*ts):
             raise ValueError("libmoeq takes CUDA tensors only")
 
 
-def _workspace(nbytes: int, device) -> torch.Tensor:
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+def _workspace(nbytes: int, device):
+    """(tensor or None, pointer or None, size argument) for a queried workspace size."""
+    if int(nbytes) == 0:
+        return None, None, None
+    ws = torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+    return ws, ws.data_ptr(), ctypes.byref(ctypes.c_size_t(ws.numel()))
 
 
 # --------------------------------------------------------------------------
@@ -155,14 +159,14 @@ def moe_route_permute(logits: torch.Tensor, x: torch.Tensor | None, k: int, chun
     L = lib()
     d = 0 if x is None else x.shape[1]
     wsb = ctypes.c_size_t(0)
-    args = lambda ws: (_p(logits), _p(x), T, E, k, d, chunk_size, _p(out.topk_idx), _p(out.gates),
-                       _p(out.expert_offsets), _p(out.active), _p(out.num_active),
-                       _p(out.chunk_offsets), _p(out.num_chunks), _p(out.perm_token),
-                       _p(out.inv_perm), _p(out.x_perm), ws, ctypes.byref(wsb), _stream(stream))
-    _check(L.moe_route_permute(*args(None)), "moe_route_permute (workspace query)")
-    ws = _workspace(wsb.value, dev)
-    wsb.value = ws.numel()
-    _check(L.moe_route_permute(*args(_p(ws))), "moe_route_permute")
+    args = lambda ws, wsz: (_p(logits), _p(x), T, E, k, d, chunk_size, _p(out.topk_idx),
+                            _p(out.gates), _p(out.expert_offsets), _p(out.active),
+                            _p(out.num_active), _p(out.chunk_offsets), _p(out.num_chunks),
+                            _p(out.perm_token), _p(out.inv_perm), _p(out.x_perm), ws, wsz,
+                            _stream(stream))
+    _check(L.moe_route_permute(*args(None, ctypes.byref(wsb))), "moe_route_permute (workspace query)")
+    ws, wsp, wsz = _workspace(wsb.value, dev)
+    _check(L.moe_route_permute(*args(wsp, wsz)), "moe_route_permute")
     return out
 
 
@@ -190,12 +194,12 @@ def moe_grouped_qgemm_fwd(a: torch.Tensor, w: QWeightT, routing: Routing, epi: i
     qw, g = qweight_c(w), routing.groups()
     wsb = ctypes.c_size_t(0)
     L = lib()
-    args = lambda ws: (_p(a), M, ctypes.byref(qw), ctypes.byref(g), _p(adapter), epi, _p(out),
-                       _p(saved) if save_gu else None, ws, ctypes.byref(wsb), _stream(stream))
-    _check(L.moe_grouped_qgemm_fwd(*args(None)), "moe_grouped_qgemm_fwd (workspace query)")
-    ws = _workspace(wsb.value, a.device)
-    wsb.value = ws.numel()
-    _check(L.moe_grouped_qgemm_fwd(*args(_p(ws))), "moe_grouped_qgemm_fwd")
+    args = lambda ws, wsz: (_p(a), M, ctypes.byref(qw), ctypes.byref(g), _p(adapter), epi,
+                            _p(out), _p(saved) if save_gu else None, ws, wsz, _stream(stream))
+    _check(L.moe_grouped_qgemm_fwd(*args(None, ctypes.byref(wsb))),
+           "moe_grouped_qgemm_fwd (workspace query)")
+    ws, wsp, wsz = _workspace(wsb.value, a.device)
+    _check(L.moe_grouped_qgemm_fwd(*args(wsp, wsz)), "moe_grouped_qgemm_fwd")
     if epi == EPI_SWIGLU:
         return out, (saved if save_gu else None)
     return out
@@ -217,13 +221,12 @@ def moe_grouped_qgemm_bwd_dx(dout: torch.Tensor, w: QWeightT, routing: Routing,
     qw, g = qweight_c(w), routing.groups()
     wsb = ctypes.c_size_t(0)
     L = lib()
-    args = lambda ws: (_p(dout), M, ctypes.byref(qw), ctypes.byref(g), epi, _p(saved_gu),
-                       _p(adapter), _p(a), _p(out), _p(d_adapter), ws, ctypes.byref(wsb),
-                       _stream(stream))
-    _check(L.moe_grouped_qgemm_bwd_dx(*args(None)), "moe_grouped_qgemm_bwd_dx (workspace query)")
-    ws = _workspace(wsb.value, dout.device)
-    wsb.value = ws.numel()
-    _check(L.moe_grouped_qgemm_bwd_dx(*args(_p(ws))), "moe_grouped_qgemm_bwd_dx")
+    args = lambda ws, wsz: (_p(dout), M, ctypes.byref(qw), ctypes.byref(g), epi, _p(saved_gu),
+                            _p(adapter), _p(a), _p(out), _p(d_adapter), ws, wsz, _stream(stream))
+    _check(L.moe_grouped_qgemm_bwd_dx(*args(None, ctypes.byref(wsb))),
+           "moe_grouped_qgemm_bwd_dx (workspace query)")
+    ws, wsp, wsz = _workspace(wsb.value, dout.device)
+    _check(L.moe_grouped_qgemm_bwd_dx(*args(wsp, wsz)), "moe_grouped_qgemm_bwd_dx")
     return (out, d_adapter) if adapter is not None else out
 
 

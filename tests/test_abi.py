@@ -58,13 +58,13 @@ def _fwd(L, a=0x80000, M=64, qw=None, g=None, adapter=None, epi=0, out=0x90000, 
 
 
 def test_fwd_workspace_query_and_validation(L):
-    wsb = ctypes.c_size_t(0)
+    wsb = ctypes.c_size_t(123)
     assert _fwd(L, wsb=wsb) == moeq.MOE_OK
-    base = wsb.value
-    assert base >= 256 and base % 256 == 0
+    assert wsb.value == 0                                            # no adapter: no workspace
     wsb2 = ctypes.c_size_t(0)
     assert _fwd(L, adapter=0xA0000, wsb=wsb2) == moeq.MOE_OK
-    assert wsb2.value >= base + 64 * 512 * 2                         # + a' rows
+    base = wsb2.value
+    assert base >= 64 * 512 * 2 and base % 256 == 0                  # a' rows
     assert _fwd(L, qw=_qw(K=96)) == 3                                # K % 64
     assert _fwd(L, qw=_qw(N=100)) == 3                               # N % 64
     assert _fwd(L, qw=_qw(fmt=7)) == 1
@@ -73,10 +73,16 @@ def test_fwd_workspace_query_and_validation(L):
     assert _fwd(L, qw=_qw(N=192), epi=1) == 3                        # SwiGLU needs N % 128
     assert _fwd(L, M=0) == 1
     small = ctypes.c_size_t(16)
-    assert _fwd(L, ws=0x100000, wsb=small) == 4                      # workspace too small
+    assert _fwd(L, adapter=0xA0000, ws=0x100000, wsb=small) == 4     # workspace too small
     ok = ctypes.c_size_t(base)
-    assert _fwd(L, ws=0x100008, wsb=ok) == 2                         # ws not 256-aligned
-    assert _fwd(L, ws=0x100000, wsb=ok, a=0x80004) == 2
+    assert _fwd(L, adapter=0xA0000, ws=0x100008, wsb=ok) == 2        # ws not 256-aligned
+    assert _fwd(L, adapter=0xA0000, ws=0x100000, wsb=ok, a=0x80004) == 2
+    # no workspace at all: fine without an adapter, an error with one
+    qw, g = _qw(), _groups()
+    assert L.moe_grouped_qgemm_fwd(0x80004, 64, ctypes.byref(qw), ctypes.byref(g), None, 0,
+                                   0x90000, None, None, None, None) == 2
+    assert L.moe_grouped_qgemm_fwd(0x80000, 64, ctypes.byref(qw), ctypes.byref(g), 0xA0000, 0,
+                                   0x90000, None, None, None, None) == 4
 
 
 def test_bwd_argument_rules(L):
