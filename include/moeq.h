@@ -146,6 +146,38 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
                              size_t* ws_bytes, void* stream);
 
 /*
+ * moe_route_permute_noalloc -- moe_route_permute for callers that cannot give
+ * the library any scratch memory. The source pages have no counterpart of
+ * this entry point; it exists for callers such as a serving runtime that
+ * reserves all device memory in one arena at start-up and allocates nothing
+ * afterwards, code that enqueues work while a CUDA graph is being captured
+ * (where cudaMalloc is not allowed), or a C host without a caching allocator,
+ * for which a cudaMalloc/cudaFree pair per call would synchronize the device.
+ *
+ * Arguments, outputs and results are those of moe_route_permute, without
+ * (ws, ws_bytes). The caller still allocates every input and output. The
+ * per-block expert histograms live in a fixed 4 MiB array inside the library
+ * (2^20 int32 entries), which every GPU that loads the library holds until
+ * the process exits. Sizes whose histograms do not fit, that is
+ * ceil(T/64) * E > 2^20, are rejected with MOE_ERR_WORKSPACE before anything
+ * is launched. The call itself never allocates or frees device memory.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. All calls on a device share the one array: calls whose kernels
+ * overlap on the GPU (different streams without ordering between them) race
+ * on it and give wrong results. Calls ordered on one stream are safe; each
+ * call rewrites the entries it reads, so leftovers of an earlier call do not
+ * matter.
+ */
+moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t T, int32_t E,
+                                     int32_t k, int64_t d, int32_t chunk_size, int32_t* topk_idx,
+                                     float* gates, int32_t* expert_offsets, int32_t* active,
+                                     int32_t* num_active, int32_t* chunk_offsets,
+                                     int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
+                                     void* x_perm, void* stream);
+
+/*
  * moe_grouped_qgemm_fwd -- forward grouped GEMM over the dequantized experts
  * (Orbit article, "Active-expert-chunked dequantization"). For every row p of
  * expert e:  acc[p] = a'[p] . W[e]^T  (fp32 accumulation on the tensor cores),

@@ -5,6 +5,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "dequant.cuh"
@@ -276,6 +277,84 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
                                   gates, expert_offsets, active, num_active, chunk_offsets,
                                   num_chunks, perm_token, inv_perm, x ? x_perm : nullptr,
                                   static_cast<int32_t*>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Routing without a caller-supplied workspace.
+//
+// Some callers cannot hand this library any scratch memory: a serving runtime
+// that reserves all of HBM in one arena at start-up and forbids device
+// allocation afterwards, code that enqueues work while a CUDA graph is being
+// captured (cudaMalloc is not capturable), or a plain C host that has no
+// caching allocator and would otherwise pay a device-wide synchronization for
+// each cudaMalloc/cudaFree pair. For them the per-block expert histograms of
+// the routing kernels live in the fixed array below, which every GPU that
+// loads the library keeps for the life of the process.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr int64_t kRouteStaticScratchInts = int64_t(1) << 20;   // 4 MiB of int32 per device
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) int32_t g_route_static_scratch[kRouteStaticScratchInts];
+
+std::mutex g_static_scratch_mutex;
+int32_t* g_static_scratch_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_route_static_scratch on the current device. In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+moe_status static_scratch_on_current_device(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mutex);
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    g_static_scratch_addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_static_scratch_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t T, int32_t E,
+                                     int32_t k, int64_t d, int32_t chunk_size, int32_t* topk_idx,
+                                     float* gates, int32_t* expert_offsets, int32_t* active,
+                                     int32_t* num_active, int32_t* chunk_offsets,
+                                     int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
+                                     void* x_perm, void* stream) {
+  if (T < 1 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || chunk_size < 1)
+    return MOE_ERR_INVALID_ARG;
+  if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  const int64_t nblk = route_num_blocks(T);
+  if (nblk * E > kRouteStaticScratchInts) return MOE_ERR_WORKSPACE;   // beyond the fixed array
+  const void* ptrs[] = {logits, topk_idx, gates, expert_offsets, active, num_active,
+                        chunk_offsets, num_chunks, perm_token, inv_perm};
+  for (const void* p : ptrs) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(p)) return MOE_ERR_MISALIGNED;
+  }
+  if (x) {
+    if (!x_perm || d < 8 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_MISALIGNED;
+  }
+  int32_t* scratch = nullptr;
+  moe_status st = static_scratch_on_current_device(&scratch);
+  if (st != MOE_OK) return st;
+  // The histogram kernel writes every entry the later kernels of this call
+  // read, so the array's leftover contents from an earlier call never matter.
+  return cuda_status(launch_route(logits, x, static_cast<int>(T), E, k, d, chunk_size, topk_idx,
+                                  gates, expert_offsets, active, num_active, chunk_offsets,
+                                  num_chunks, perm_token, inv_perm, x ? x_perm : nullptr, scratch,
+                                  static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,

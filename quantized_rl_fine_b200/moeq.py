@@ -29,7 +29,7 @@ FMT = {"int4": W_INT4, "mxfp4": W_MXFP4}
 EPI_NONE, EPI_SWIGLU, EPI_SWIGLU_BWD = 0, 1, 2
 DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_OFFSETS = 0, 1, 2
 
-EXPORTED = ("moe_route_permute", "moe_grouped_qgemm_fwd", "moe_grouped_qgemm_bwd_dx",
+EXPORTED = ("moe_route_permute", "moe_route_permute_noalloc", "moe_grouped_qgemm_fwd", "moe_grouped_qgemm_bwd_dx",
             "moe_unpermute_combine", "moe_get_device_error", "moe_status_string",
             "moe_abi_version", "moe_test_dequant", "moe_test_set_wait_budget")
 
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)
     L.moe_route_permute.argtypes = [vp, vp, i64, i32, i32, i64, i32, vp, vp, vp, vp, vp, vp, vp,
                                     vp, vp, vp, vp, sz, vp]
+    L.moe_route_permute_noalloc.argtypes = [vp, vp, i64, i32, i32, i64, i32, vp, vp, vp, vp, vp,
+                                            vp, vp, vp, vp, vp, vp]
     L.moe_grouped_qgemm_fwd.argtypes = [vp, i64, ctypes.POINTER(QWeightC), ctypes.POINTER(GroupsC),
                                         vp, i32, vp, vp, vp, sz, vp]
     L.moe_grouped_qgemm_bwd_dx.argtypes = [vp, i64, ctypes.POINTER(QWeightC),
