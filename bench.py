@@ -352,7 +352,7 @@ def _step_fn(cfg, chunk):
 
 
 def _launches_per_step(cfg):
-    route = 3
+    route = 4
     if not cfg.swiglu:
         return route + 1
     n = route + 2 + 1                           # gate/up, down, combine
@@ -363,6 +363,12 @@ def _launches_per_step(cfg):
         if cfg.adapter:
             n += 2                              # adapter backward (dx, dR)
     return n
+
+
+def _check_device(moeq, phase):
+    code = moeq.moe_get_device_error()
+    if code != 0:
+        raise SystemExit(f"device error word {code} after the {phase}: results are not valid")
 
 
 def run_ours(args, cfg):
@@ -432,7 +438,7 @@ def run_ours(args, cfg):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
     ms_per_step = ms / args.steps
-    assert moeq.moe_get_device_error() == 0
+    _check_device(moeq, "timed steps")
 
     # ---------------------------------------------------------------- dominant kernel alone
     from quantized_rl_fine_b200 import layer
@@ -459,6 +465,7 @@ def run_ours(args, cfg):
     kb.record(stream)
     torch.cuda.synchronize()
     k_ms = ka.elapsed_time(kb) / n_k
+    _check_device(moeq, "grouped GEMM alone")
 
     # ---------------------------------------------------------------- end to end via host buffers
     host = []
@@ -498,7 +505,7 @@ def run_ours(args, cfg):
         tt = torch.tensor([e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e_ms = float(tt.item())
-    assert moeq.moe_get_device_error() == 0
+    _check_device(moeq, "end-to-end steps")
 
     # ---------------------------------------------------------------- report
     del graphs, gemm_graphs

@@ -62,19 +62,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D tiled tensor map over a row-major [rows][cols] array.
-bool make_map_2d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esize,
-                 uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-                 CUtensorMapSwizzle sw) {
+// 3-D tiled tensor map: extents dims[0..2] (dims[0] contiguous), byte strides
+// of dims 1 and 2, box extents box[0..2]. A 2-D map is dims[2] = 1.
+bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, const uint64_t dims[3],
+                 const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle sw) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t b[3] = {box[0], box[1], box[2]};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), d, st, b, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -94,17 +93,17 @@ int max_smem_optin() {
 }
 
 // Token rows per tile from the mean rows per expert: ~1.4x the mean split
-// into as few tiles of <= 256 as possible, rounded up to a multiple of 16.
-int choose_bn(int64_t M, int E) {
+// into as few tiles of <= max_bn as possible, rounded up to a multiple of 16.
+int choose_bn(int64_t M, int E, int max_bn) {
   if (const char* env = getenv("MOEQ_BN")) {
     const int v = atoi(env);
-    if (v >= 16 && v <= 256 && v % 16 == 0) return v;
+    if (v >= 16 && v <= max_bn && v % 16 == 0) return v;
   }
   const double mean = static_cast<double>(M) / std::max(1, E);
   const double want = std::max(1.0, 1.4 * mean);
-  const int tiles = static_cast<int>((want + 255.0) / 256.0);
+  const int tiles = static_cast<int>((want + max_bn - 1.0) / max_bn);
   int bn = static_cast<int>((want / tiles + 15.0) / 16.0) * 16;
-  return std::min(256, std::max(16, bn));
+  return std::min(max_bn, std::max(16, bn));
 }
 
 int next_pow2(int x) {
@@ -131,24 +130,44 @@ moe_status check_groups(const moe_groups* g, int E) {
 }
 
 struct GemmPlan {
-  int BN, stages, grid, n_ftiles;
+  int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers;
   uint32_t stage_bytes;
   size_t smem;
 };
 
 // F: output features; tile_f: output features per tile (128, or 64 for the
 // SwiGLU forward, whose tile holds 64 gate and the 64 matching up rows).
-GemmPlan plan_gemm(int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
+// Tensor memory (512 columns) holds n_issuers partial accumulators of
+// acc_cols columns each and, in the forward kernels, the A stages (64
+// columns per 128-wide fill). Forward token tiles are capped at 160 rows so
+// that at least four A stages fit; backward tiles (A in shared memory) go up
+// to 256.
+GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
   GemmPlan pl;
-  pl.BN = choose_bn(M, w->E);
-  pl.stage_bytes = gemm_stage_bytes(pl.BN, fmt);
+  pl.BN = choose_bn(M, w->E, mode == kModeFwd ? 160 : 256);
+  pl.acc_cols = (pl.BN + 31) / 32 * 32;
+  pl.stage_bytes = gemm_stage_bytes(mode, pl.BN, fmt);
+  if (mode == kModeFwd) {
+    // A stage of a 128-wide fill: 64 columns; keep at least four of them.
+    pl.n_issuers = std::max(1, std::min(3, (512 - 4 * 64) / pl.acc_cols));
+    pl.a_stages = std::min(8, (512 - pl.n_issuers * pl.acc_cols) / 64);
+    pl.tmem_cols = 512;
+  } else {
+    pl.n_issuers = std::max(1, std::min(3, 512 / pl.acc_cols));
+    pl.tmem_cols = next_pow2(pl.n_issuers * pl.acc_cols);
+  }
+  // As many shared-memory fills as fit (at most 16): a deep ring hides the
+  // latency of the weight stream.
   const int avail = max_smem_optin();
-  int stages = 8;
-  while (stages > 2 &&
-         static_cast<int>(stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, w->E)) > avail)
-    --stages;
+  int stages = 16;
+  auto fits = [&](int s) {
+    const int sa = (mode == kModeFwd) ? pl.a_stages : s;
+    return static_cast<int>(s * pl.stage_bytes + gemm_fixed_smem_bytes(s, sa, w->E)) <= avail;
+  };
+  while (stages > 4 && !fits(stages)) --stages;
   pl.stages = stages;
-  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, w->E);
+  if (mode != kModeFwd) pl.a_stages = stages;
+  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
   pl.n_ftiles = (F + tile_f - 1) / tile_f;
   const int64_t bound = static_cast<int64_t>(pl.n_ftiles) *
                         (std::min<int64_t>(w->E, M) + (M + pl.BN - 1) / pl.BN);
@@ -183,26 +202,52 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   const int R = (mode == kModeFwd) ? w->K : w->N;
   CUtensorMap tb, tw, ts;
   const bool int4 = w->fmt == MOE_W_INT4_G32_BF16;
-  if (!make_map_2d(&tb, bmat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, M, 64, pl.BN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-    return MOE_ERR_CUDA;
-  if (mode == kModeFwd) {
-    if (!make_map_2d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K / 2,
-                     static_cast<uint64_t>(w->E) * w->N, 32, 64, CU_TENSOR_MAP_SWIZZLE_32B))
+  const uint64_t esz = int4 ? 2 : 1;
+  const CUtensorMapDataType sdt = int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint64_t E = w->E, N = w->N, K = w->K;
+  const uint32_t chunks = (mode == kModeFwd) ? 2 : 1;      // 64-element K chunks per fill
+  {  // token rows: [M][R] BF16 viewed as (64, M, R/64) -> smem [chunk][BN rows][64]
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(M), static_cast<uint64_t>(R) / 64};
+    const uint64_t strides[2] = {static_cast<uint64_t>(R) * 2, 128};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(pl.BN), chunks};
+    if (!make_map_3d(&tb, bmat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
       return MOE_ERR_CUDA;
-    if (!make_map_2d(&ts, w->scales,
-                     int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                     int4 ? 2 : 1, w->N, static_cast<uint64_t>(w->E) * (w->K / 32), 64, 2,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
+  }
+  if (mode == kModeFwd && epi == MOE_EPI_SWIGLU) {
+    // packed [E][N][K/2] as [2E][N/2][K/2]: one box brings 64 gate and the 64 up rows
+    const uint64_t wd[3] = {K / 2, N / 2, 2 * E};
+    const uint64_t ws[2] = {K / 2, (N / 2) * (K / 2)};
+    const uint32_t wb[3] = {64, 64, 2};
+    // scales [E][K/32][N] as [E*K/32][2][N/2] -> smem [4 groups][2 halves][64]
+    const uint64_t sd[3] = {N / 2, 2, E * (K / 32)};
+    const uint64_t ss[2] = {(N / 2) * esz, N * esz};
+    const uint32_t sb[3] = {64, 2, 4};
+    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return MOE_ERR_CUDA;
+  } else if (mode == kModeFwd) {
+    const uint64_t wd[3] = {K / 2, E * N, 1};
+    const uint64_t ws[2] = {K / 2, E * N * (K / 2)};
+    const uint32_t wb[3] = {64, 128, 1};
+    const uint64_t sd[3] = {N, E * (K / 32), 1};
+    const uint64_t ss[2] = {N * esz, E * (K / 32) * N * esz};
+    const uint32_t sb[3] = {128, 4, 1};
+    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
   } else {
-    if (!make_map_2d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->K / 2,
-                     static_cast<uint64_t>(w->E) * w->N, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B))
-      return MOE_ERR_CUDA;
-    if (!make_map_2d(&ts, w->scales,
-                     int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                     int4 ? 2 : 1, w->N, static_cast<uint64_t>(w->E) * (w->K / 32), 64, 4,
-                     CU_TENSOR_MAP_SWIZZLE_NONE))
+    const uint64_t wd[3] = {K / 2, E * N, 1};
+    const uint64_t ws[2] = {K / 2, E * N * (K / 2)};
+    const uint32_t wb[3] = {64, 64, 1};
+    const uint64_t sd[3] = {N, E * (K / 32), 1};
+    const uint64_t ss[2] = {N * esz, E * (K / 32) * N * esz};
+    const uint32_t sb[3] = {64, 4, 1};
+    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb,
+                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
   }
   GemmArgs p;
@@ -215,11 +260,13 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   p.M = static_cast<int32_t>(M);
   p.BN = pl.BN;
   p.n_ftiles = pl.n_ftiles;
-  p.acc_cols = (pl.BN + 31) / 32 * 32;
-  p.tmem_cols = next_pow2(2 * p.acc_cols);
+  p.n_issuers = pl.n_issuers;
+  p.acc_cols = pl.acc_cols;
+  p.tmem_cols = pl.tmem_cols;
   p.F = F;
   p.R = R;
   p.stages = pl.stages;
+  p.a_stages = pl.a_stages;
   p.stage_bytes = pl.stage_bytes;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ldo = ldo;
@@ -366,7 +413,7 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
   if (epi != MOE_EPI_NONE && epi != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (epi == MOE_EPI_SWIGLU && w->N % 128 != 0) return MOE_ERR_UNSUPPORTED;
   const int F = (epi == MOE_EPI_SWIGLU) ? w->N / 2 : w->N;
-  const GemmPlan pl = plan_gemm(M, w, F, epi == MOE_EPI_SWIGLU ? 64 : 128, w->fmt);
+  const GemmPlan pl = plan_gemm(kModeFwd, M, w, F, epi == MOE_EPI_SWIGLU ? 64 : 128, w->fmt);
   const size_t need = adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
   if ((st = check_workspace(ws, ws_bytes, need)) != MOE_OK) return st;
   if (!ws && ws_bytes) return MOE_OK;   // size query
@@ -400,7 +447,7 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
   if (with_adapter && (epi != MOE_EPI_NONE || !a || !d_adapter)) return MOE_ERR_INVALID_ARG;
   if (!with_adapter && (a || d_adapter)) return MOE_ERR_INVALID_ARG;
   if (epi == MOE_EPI_SWIGLU_BWD && !saved_gu) return MOE_ERR_INVALID_ARG;
-  const GemmPlan pl = plan_gemm(M, w, w->K, 128, w->fmt);
+  const GemmPlan pl = plan_gemm(kModeBwd, M, w, w->K, 128, w->fmt);
   const size_t need = with_adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
   if ((st = check_workspace(ws, ws_bytes, need)) != MOE_OK) return st;
   if (!ws && ws_bytes) return MOE_OK;   // size query

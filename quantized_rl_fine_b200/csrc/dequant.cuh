@@ -24,9 +24,17 @@ __device__ __forceinline__ uint32_t pair_select(int p) {
   return static_cast<uint32_t>(p | (p << 4) | ((4 + p) << 8) | ((4 + p) << 12));
 }
 
+// w >> 4 as a multiply-high, so the shift runs on the FMA pipe and leaves the
+// integer ALU pipe (which carries the byte permutes and logic ops) free.
+__device__ __forceinline__ uint32_t shr4(uint32_t w) {
+  uint32_t r;
+  asm("mul.hi.u32 %0, %1, 268435456;" : "=r"(r) : "r"(w));
+  return r;
+}
+
 // 8 INT4 codes of one 32-bit word -> 4 BF16 pairs, scale pair s2 = {s, s}.
 __device__ __forceinline__ void dequant8_int4(uint32_t w, uint32_t s2, uint32_t (&o)[4]) {
-  const uint32_t odd = w >> 4;
+  const uint32_t odd = shr4(w);
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     uint32_t t = prmt(w, odd, pair_select(p));
@@ -57,9 +65,11 @@ __device__ __forceinline__ MxScale mx_scale(uint32_t X) {
   return s;
 }
 
-// 8 E2M1 codes of one 32-bit word -> 4 BF16 pairs.
+// 8 E2M1 codes of one 32-bit word -> 4 BF16 pairs; TWO selects the second
+// multiply (exponents above 128).
+template <bool TWO>
 __device__ __forceinline__ void dequant8_mxfp4(uint32_t w, const MxScale& s, uint32_t (&o)[4]) {
-  const uint32_t odd = w >> 4;
+  const uint32_t odd = shr4(w);
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const uint32_t t = prmt(w, odd, pair_select(p)) & 0x000F000Fu;   // {c_even, c_odd}
@@ -67,7 +77,7 @@ __device__ __forceinline__ void dequant8_mxfp4(uint32_t w, const MxScale& s, uin
     // (bits 28..31 for the upper half); the mask drops the spare copies.
     const uint32_t v = (t * 0x1040u) & 0x81C081C0u;
     uint32_t r = bf16x2_mul(v, s.a);
-    if (s.two) r = bf16x2_mul(r, s.b);
+    if constexpr (TWO) r = bf16x2_mul(r, s.b);
     o[p] = r;
   }
 }
@@ -88,13 +98,25 @@ __device__ __forceinline__ void dequant32(const uint4& pk, uint32_t scale_bits, 
       for (int j = 0; j < 4; ++j) o[4 * i + j] = q[j];
     }
   } else {
+    // One branch per 32-element group: the second multiply is needed only for
+    // exponents above 128, which real weights never use.
     const MxScale s = mx_scale(scale_bits);
+    if (!s.two) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint32_t q[4];
-      dequant8_mxfp4(words[i], s, q);
+      for (int i = 0; i < 4; ++i) {
+        uint32_t q[4];
+        dequant8_mxfp4<false>(words[i], s, q);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) o[4 * i + j] = q[j];
+        for (int j = 0; j < 4; ++j) o[4 * i + j] = q[j];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t q[4];
+        dequant8_mxfp4<true>(words[i], s, q);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[4 * i + j] = q[j];
+      }
     }
   }
 }

@@ -35,10 +35,11 @@ namespace moeq {
 namespace {
 
 constexpr int kThreads = kGemmThreads;
-constexpr int kStageK = 64;            // reduction elements per pipeline stage
+constexpr int kDqWarp0 = 4;                              // first dequant warp
+constexpr int kEpiWarp0 = kDqWarp0 + 4 * kDqGroups;      // first epilogue warp
+static_assert(kThreads == 32 * (kEpiWarp0 + 4), "warp roles must fill the CTA");
 constexpr int kTileF = 128;            // output features per tile (MMA M)
-constexpr uint32_t kABytes = kTileF * kStageK * 2;   // 16 KiB dequantized tile
-constexpr uint32_t kWqBytes = 4096;    // packed weights of one stage
+constexpr uint32_t kABytes = kTileF * 64 * 2;   // 16 KiB dequantized A tile (backward fill)
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -69,9 +70,9 @@ __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
 
 // A wait used only while shutting down: bounded, ignores the abort flag.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  const long long budget = g_wait_budget;
+  const long long budget = kDefaultWaitBudget;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) {
     if (clock64() - t0 > budget) {
       raise_device_error(MOE_DEVERR_WAIT_TIMEOUT);
       return;
@@ -165,8 +166,16 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_wq,
                      const __grid_constant__ CUtensorMap tm_sc, const GemmArgs p) {
   constexpr uint32_t kScEl = (FMT == MOE_W_INT4_G32_BF16) ? 2 : 1;
-  constexpr uint32_t kScBytes = 256 * kScEl;   // scales of one stage
   constexpr bool kGluRows = (MODE == kModeFwd && EPI == MOE_EPI_SWIGLU);
+  // Forward: fills of 128 reduction elements; the dequantized A tile goes to
+  // tensor memory (two 32-column sub-stages per fill). Backward: fills of 64,
+  // A in a 128B-swizzled MN-major shared-memory tile.
+  constexpr bool kTmemA = (MODE == kModeFwd);
+  constexpr int kFillK = kTmemA ? 128 : 64;
+  constexpr uint32_t kSmemA = kTmemA ? 0u : kABytes;
+  constexpr uint32_t kWqFill = kTmemA ? 8192u : 4096u;            // packed bytes per fill
+  constexpr uint32_t kScFill = (kTmemA ? 512u : 256u) * kScEl;    // scale bytes per fill
+  constexpr int kBChunks = kFillK / 64;                           // 128-byte K chunks of B
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -175,23 +184,31 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
 
   const int S = p.stages;
   const uint32_t stage_bytes = p.stage_bytes;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.BN) * 128u;
-  // One stage: [A 16 KiB][B BN*128][packed 4 KiB][scales 256 or 512 B]
-  auto A_at = [&](int s) { return base + s * stage_bytes; };
-  auto B_at = [&](int s) { return base + s * stage_bytes + kABytes; };
-  auto W_at = [&](int s) { return base + s * stage_bytes + kABytes + b_bytes; };
-  auto S_at = [&](int s) { return base + s * stage_bytes + kABytes + b_bytes + kWqBytes; };
+  const uint32_t b_chunk = static_cast<uint32_t>(p.BN) * 128u;   // one [BN][64] BF16 chunk
+  const uint32_t b_bytes = b_chunk * kBChunks;
+  // One stage: [B kBChunks x BN*128][A 16 KiB (backward only)][packed][scales]
+  auto B_at = [&](int s) { return base + s * stage_bytes; };
+  auto A_at = [&](int s) { return base + s * stage_bytes + b_bytes; };
+  auto W_at = [&](int s) { return base + s * stage_bytes + b_bytes + kSmemA; };
+  auto S_at = [&](int s) { return base + s * stage_bytes + b_bytes + kSmemA + kWqFill; };
+  // Two rings: S shared-memory fills (TMA) and SA A stages. In the forward
+  // kernels the A stages live in tensor memory and may be fewer than the
+  // fills; in the backward kernels the A tile is part of the fill (SA = S).
+  const int SA = p.a_stages;
   const uint32_t bars = base + S * stage_bytes;
   auto full_tma = [&](int s) { return bars + 8u * s; };
-  auto full_a = [&](int s) { return bars + 8u * (S + s); };
-  auto empty = [&](int s) { return bars + 8u * (2 * S + s); };
-  auto acc_full = [&](int b) { return bars + 8u * (3 * S + b); };
-  auto acc_empty = [&](int b) { return bars + 8u * (3 * S + 2 + b); };
-  const uint32_t drain_bar = bars + 8u * (3 * S + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (3 * S + 5));
+  auto empty = [&](int s) { return bars + 8u * (S + s); };
+  auto full_a = [&](int s) { return bars + 8u * (2 * S + s); };
+  auto a_free = [&](int s) { return bars + 8u * (2 * S + SA + s); };
+  const uint32_t acc_full = bars + 8u * (2 * S + 2 * SA);
+  const uint32_t acc_empty = bars + 8u * (2 * S + 2 * SA + 1);
+  const uint32_t drain_bar = bars + 8u * (2 * S + 2 * SA + 2);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (2 * S + 2 * SA + 3));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* warp_tot = reinterpret_cast<int32_t*>(tmem_slot + 4);          // [32]
   int32_t* tile_start = warp_tot + 32;                                      // [E + 1]
+  // Epilogue staging: one 4 KiB block per epilogue warp (16 token rows x 64 BF16 used).
+  const uint32_t stg_base = (smem_u32(tile_start + p.E + 1) + 127u) & ~127u;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -199,14 +216,15 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full_tma(s), 1);
-      mbar_init(full_a(s), 4);
       mbar_init(empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full(b), 1);
-      mbar_init(acc_empty(b), 4);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(full_a(s), 4);
+      mbar_init(a_free(s), 1);
     }
-    mbar_init(drain_bar, 1);
+    mbar_init(acc_full, p.n_issuers);
+    mbar_init(acc_empty, 4);
+    mbar_init(drain_bar, p.n_issuers);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -223,15 +241,20 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
 
   const int A = build_tile_list(p, tile_start, warp_tot);
   const int total = tile_start[A];
-  const int nkb = p.R / kStageK;
+  const int nkb = (p.R + kFillK - 1) / kFillK;   // forward K % 128 may be 64: zero tail
   const int N = p.N, K = p.K;
+  // Tensor-memory columns: [partial accumulator 0 .. NI-1][A stage 0 .. S-1 (forward)].
+  const int NI = p.n_issuers;
+  const uint32_t a_col0 = static_cast<uint32_t>(NI * p.acc_cols);
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const uint64_t keep = l2_policy_evict_last();
-      const uint64_t stream_once = l2_policy_evict_first();
-      const uint32_t tx = b_bytes + kWqBytes + kScBytes;
+    // Lanes 0-2 issue the fill's three bulk tensor copies in one instruction:
+    // lane 0 the token rows, lane 1 the packed weights, lane 2 the group scales.
+    if (lane < 3) {
+      const uint64_t policy = (lane == 0) ? l2_policy_evict_last() : l2_policy_evict_first();
+      const CUtensorMap* map = (lane == 0) ? &tm_b : (lane == 1) ? &tm_wq : &tm_sc;
+      const uint32_t tx = b_bytes + kWqFill + kScFill;
       int st = 0;
       uint32_t ph = 0;
       long long fills = 0;
@@ -239,123 +262,193 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(p, tile_start, A, t);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_tma(st), tx);
-          tma_load_2d_hint(B_at(st), &tm_b, full_tma(st), kb * kStageK, tl.row0, keep);
-          if constexpr (MODE == kModeFwd) {
-            int fa, fb;
-            if constexpr (EPI == MOE_EPI_SWIGLU) {
-              fa = tl.ft * 64;            // gate rows
-              fb = N / 2 + tl.ft * 64;    // the matching up rows
-            } else {
-              fa = tl.ft * kTileF;
-              fb = fa + 64;
+          // Lane 0 waits; the three lanes leave or go on together.
+          int got = 1;
+          if (lane == 0) got = mbar_wait(empty(st), ph ^ 1u, abort_flag) ? 1 : 0;
+          got = __shfl_sync(0x7u, got, 0);
+          if (!got) { ok = false; break; }
+          if (lane == 0) mbar_arrive_expect_tx(full_tma(st), tx);
+          uint32_t dst;
+          int c0, c1, c2;
+          if (lane == 0) {                       // rows x [kFillK] BF16
+            dst = B_at(st);
+            c0 = 0;
+            c1 = tl.row0;
+            c2 = kb * kBChunks;
+          } else if constexpr (MODE == kModeFwd) {
+            if (lane == 1) {                     // packed: [2 halves or 1][rows][64 B]
+              dst = W_at(st);
+              c0 = kb * 64;
+              if constexpr (EPI == MOE_EPI_SWIGLU) { c1 = tl.ft * 64; c2 = 2 * tl.e; }
+              else { c1 = tl.e * N + tl.ft * kTileF; c2 = 0; }
+            } else {                             // scales: [4 groups][128 rows]
+              dst = S_at(st);
+              if constexpr (EPI == MOE_EPI_SWIGLU) { c0 = tl.ft * 64; c1 = 0; c2 = tl.e * (K / 32) + kb * 4; }
+              else { c0 = tl.ft * kTileF; c1 = tl.e * (K / 32) + kb * 4; c2 = 0; }
             }
-            const int g0 = tl.e * (K / 32) + kb * 2;
-            tma_load_2d_hint(W_at(st), &tm_wq, full_tma(st), kb * 32, tl.e * N + fa, stream_once);
-            tma_load_2d_hint(W_at(st) + 2048, &tm_wq, full_tma(st), kb * 32, tl.e * N + fb,
-                             stream_once);
-            tma_load_2d_hint(S_at(st), &tm_sc, full_tma(st), fa, g0, stream_once);
-            tma_load_2d_hint(S_at(st) + 128 * kScEl, &tm_sc, full_tma(st), fb, g0, stream_once);
           } else {
-            tma_load_2d_hint(W_at(st), &tm_wq, full_tma(st), tl.ft * 64, tl.e * N + kb * kStageK,
-                             stream_once);
-            tma_load_2d_hint(S_at(st), &tm_sc, full_tma(st), kb * kStageK,
-                             tl.e * (K / 32) + tl.ft * 4, stream_once);
+            if (lane == 1) {                     // packed: [64 rows][64 B]
+              dst = W_at(st);
+              c0 = tl.ft * 64;
+              c1 = tl.e * N + kb * kFillK;
+              c2 = 0;
+            } else {                             // scales: [4 groups][64 rows]
+              dst = S_at(st);
+              c0 = kb * kFillK;
+              c1 = tl.e * (K / 32) + tl.ft * 4;
+              c2 = 0;
+            }
           }
+          __syncwarp(0x7u);
+          tma_load_3d_hint(dst, map, full_tma(st), c0, c1, c2, policy);
           ++fills;
           if (++st == S) { st = 0; ph ^= 1u; }
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         // Let every issued copy land before the CTA can exit.
         const long long first = fills > S ? fills - S : 0;
         for (long long f = first; f < fills; ++f)
           mbar_drain(full_tma(static_cast<int>(f % S)), static_cast<uint32_t>((f / S) & 1));
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 1 && warp <= NI) {
+    // ------------------------------------------------------------ MMA issuers
+    // One thread issuing tcgen05.mma sustains only about one instruction per
+    // ~100 cycles whatever N is, so the K loop of a tile is split among NI
+    // issuing warps: issuer j takes the fills kb with kb % NI == j into its own
+    // partial accumulator; the epilogue adds the partials in a fixed order.
     if (lane == 0) {
+      const int j = warp - 1;
       const uint32_t idesc = idesc_bf16_f32(kTileF, p.BN, MODE == kModeBwd ? 1u : 0u, 0u);
-      int st = 0;
-      uint32_t ph = 0;
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(j * p.acc_cols);
+      int st = 0, sa = 0;
+      uint32_t ph = 0, pha = 0;
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const int buf = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait(acc_empty(buf), aph ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(acc_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * p.acc_cols);
+        uint32_t acc = 0;
+        int r = 0;                            // kb % NI
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(full_tma(st), ph, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(full_a(st), ph, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kStageK / 16; ++kk) {
-            uint64_t adesc;
-            if constexpr (MODE == kModeFwd) {
-              adesc = smem_desc_sw128(A_at(st) + kk * 32, 16, 1024);
+          if (r == j) {
+            if (!mbar_wait(full_a(sa), pha, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
+            if constexpr (kTmemA) {
+              // A stage st: 128 lanes x 64 columns (two BF16 per column): K=16 = 8 columns.
+              const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * 64);
+              const uint64_t b1 = b0 + (b_chunk >> 4);
+              mma_bf16_ts(d_tmem, a0, b0, idesc, acc);
+              mma_bf16_ts(d_tmem, a0 + 8, b0 + 2, idesc, 1u);
+              mma_bf16_ts(d_tmem, a0 + 16, b0 + 4, idesc, 1u);
+              mma_bf16_ts(d_tmem, a0 + 24, b0 + 6, idesc, 1u);
+              mma_bf16_ts(d_tmem, a0 + 32, b1, idesc, 1u);
+              mma_bf16_ts(d_tmem, a0 + 40, b1 + 2, idesc, 1u);
+              mma_bf16_ts(d_tmem, a0 + 48, b1 + 4, idesc, 1u);
+              mma_bf16_ts(d_tmem, a0 + 56, b1 + 6, idesc, 1u);
             } else {
-              adesc = smem_desc_sw128(A_at(st) + kk * 2048, 8192, 1024);
+              const uint64_t a0 = smem_desc_sw128(A_at(st), 8192, 1024);
+              mma_bf16_ss(d_tmem, a0, b0, idesc, acc);
+              mma_bf16_ss(d_tmem, a0 + 128, b0 + 2, idesc, 1u);
+              mma_bf16_ss(d_tmem, a0 + 256, b0 + 4, idesc, 1u);
+              mma_bf16_ss(d_tmem, a0 + 384, b0 + 6, idesc, 1u);
             }
-            const uint64_t bdesc = smem_desc_sw128(B_at(st) + kk * 32, 16, 1024);
-            mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+            acc = 1u;
+            mma_commit(empty(st));
+            if constexpr (kTmemA) mma_commit(a_free(sa));
           }
-          mma_commit(empty(st));
+          if (++r == NI) r = 0;
           if (++st == S) { st = 0; ph ^= 1u; }
+          if (++sa == SA) { sa = 0; pha ^= 1u; }
         }
-        if (ok) mma_commit(acc_full(buf));
+        if (ok) mma_commit(acc_full);         // arrives even when this issuer had no fill
       }
       // All MMAs of this CTA done before tensor memory is released.
       mma_commit(drain_bar);
       mbar_drain(drain_bar, 0);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + 4 * kDqGroups) {
     // ------------------------------------------------------------ dequantizers
-    const int i = threadIdx.x - 128;   // 0..127
-    // Forward: thread i writes A row i (one output feature). With SwiGLU the
-    // rows interleave gate and up: row 2j <- gate row j (packed row j), row
-    // 2j+1 <- up row j (packed row 64 + j).
-    const int src = kGluRows ? ((i & 1) ? 64 + (i >> 1) : (i >> 1)) : i;
-    int st = 0;
-    uint32_t ph = 0;
+    // kDqGroups warpgroups take the fills in turn (fill f goes to group f % kDqGroups).
+    const int grp = (warp - kDqWarp0) >> 2;
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    const int i = q * 32 + lane;            // A row (forward) / thread slot (backward)
+    // Forward: A row i is one output feature. With SwiGLU each warp's 32 rows
+    // hold 16 gate rows (lanes 0-15: packed rows 16q + l) and the 16 matching
+    // up rows (lanes 16-31: packed rows 64 + 16q + l - 16), so every 8-lane
+    // phase of a 128-bit shared load touches 8 distinct swizzle slots.
+    const int src = kGluRows ? ((lane < 16) ? (16 * q + lane) : (64 + 16 * q + lane - 16)) : i;
+    // Fill f of the CTA uses stage f % S with parity (f / S) & 1; this group
+    // owns fills grp, grp + kDqGroups, ... and steps its stage and parity
+    // incrementally (kDqGroups < S).
+    int turn = 0;                           // f % kDqGroups
+    int st = grp, sa = grp;                 // fill ring and A ring positions of the next own fill
+    uint32_t ph = 0, pha = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!mbar_wait(full_tma(st), ph, abort_flag)) { ok = false; break; }
-        const uint32_t wq = W_at(st);
-        const uint32_t sc = S_at(st);
-        const uint32_t a_st = A_at(st);
+        const bool mine = (turn == grp);
+        if (++turn == kDqGroups) turn = 0;
+        if (!mine) continue;
+        const int cur = st, cur_a = sa;
+        const uint32_t cur_ph = ph, cur_pha = pha;
+        const int kb_cur = kb;
+        st += kDqGroups;
+        if (st >= S) { st -= S; ph ^= 1u; }
+        sa += kDqGroups;
+        if (sa >= SA) { sa -= SA; pha ^= 1u; }
+        if (!mbar_wait(full_tma(cur), cur_ph, abort_flag)) { ok = false; break; }
+        // Forward: the A stage must have been released by the MMAs of the
+        // fill that used it SA fills ago.
+        if (kTmemA && !mbar_wait(a_free(cur_a), cur_pha ^ 1u, abort_flag)) { ok = false; break; }
+        const uint32_t wq = W_at(cur);
+        const uint32_t sc = S_at(cur);
         if constexpr (MODE == kModeFwd) {
-          // Packed rows are 32 bytes with the TMA 32-byte swizzle (16-byte chunk
-          // index ^= row bit 2). Scales: two boxes [2 groups][64 rows].
+          // Packed rows are 64 bytes with the TMA 64-byte swizzle (16-byte chunk
+          // index ^= (row >> 1) & 3). Scales: [4 groups][128 rows].
+          const uint32_t prow = wq + src * 64;
+          const uint32_t sw = (src >> 1) & 3;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint4 pk = lds128(wq + src * 32 + ((h ^ ((src >> 2) & 1)) << 4));
-            const uint32_t soff = (src >> 6) * 128 + h * 64 + (src & 63);
-            const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
-                                                                : lds_u8(sc + soff);
-            uint32_t o[16];
-            dequant32<FMT>(pk, sbits, o);
-            // K-major, 128B swizzle: row i at (i/8)*1024 + (i%8)*128, chunk c ^ (i%8).
-            const uint32_t rowb = a_st + (i >> 3) * 1024 + (i & 7) * 128;
+          for (int h2 = 0; h2 < 2; ++h2) {
+            uint32_t o[32];
+            // A half fill past the reduction length (K % 128 == 64) is zero, so
+            // neither the zero-filled codes nor a foreign scale can reach the MMA.
+            if (kb_cur * kFillK + h2 * 64 >= p.R) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint32_t chunk = (h * 4 + c) ^ (i & 7);
-              sts128(rowb + (chunk << 4), o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+              for (int jj = 0; jj < 32; ++jj) o[jj] = 0u;
+            } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int c = 2 * h2 + h;     // 32-element group of this fill
+              const uint4 pk = lds128(prow + ((c ^ sw) << 4));
+              const uint32_t soff = c * 128 + src;
+              const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
+                                                                  : lds_u8(sc + soff);
+              uint32_t oh[16];
+              dequant32<FMT>(pk, sbits, oh);
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) o[16 * h + jj] = oh[jj];
             }
+            }
+            // Lane i of the A sub-stage: 32 columns = 64 BF16 along K, low half = even k.
+            tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a_col0 +
+                                   static_cast<uint32_t>(cur_a * 64 + h2 * 32),
+                               o);
           }
+          tmem_wait_st();
+          tc_fence_before();
         } else {
           // Thread = (reduction row r, feature half hf): 64 features = 2 groups.
           // Packed rows are 64 bytes with the TMA 64-byte swizzle (chunk ^= (r >> 1) & 3).
-          // Scales: one box [4 groups][64 rows].
+          // Scales: [4 groups][64 rows].
+          const uint32_t a_st = A_at(cur);
           const int r = i & 63;
           const int hf = i >> 6;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int c = 2 * hf + j;
+          for (int jh = 0; jh < 2; ++jh) {
+            const int c = 2 * hf + jh;
             const uint4 pk = lds128(wq + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
             const uint32_t soff = c * 64 + r;
             const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
@@ -367,89 +460,135 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             const uint32_t rowb = a_st + hf * 8192 + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
-              const uint32_t chunk = (4 * j + w) ^ (r & 7);
+              const uint32_t chunk = (4 * jh + w) ^ (r & 7);
               sts128(rowb + (chunk << 4), o[4 * w], o[4 * w + 1], o[4 * w + 2], o[4 * w + 3]);
             }
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(full_a(st));
-        if (++st == S) { st = 0; ph ^= 1u; }
+        if (lane == 0) mbar_arrive(full_a(cur_a));
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
+    // Sums the partial accumulators (fixed order), converts to BF16, stages 32
+    // token rows at a time in this warp's shared block and writes them with
+    // 16-byte stores, only for rows that belong to the tile's expert.
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int fr = q * 32 + lane;           // accumulator row = tile feature
+    const uint32_t stg = stg_base + static_cast<uint32_t>(q) * 4096u;
+    uint16_t* stg_ptr = reinterpret_cast<uint16_t*>(gbase + (stg - base));
+    const int nacc = NI < nkb ? NI : nkb;
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const Tile tl = decode_tile(p, tile_start, A, t);
-      const int buf = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
-      if (!mbar_wait(acc_full(buf), aph, abort_flag)) break;
+      if (!mbar_wait(acc_full, static_cast<uint32_t>(it & 1), abort_flag)) break;
       tc_fence_after();
-      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                            static_cast<uint32_t>(buf * p.acc_cols);
-      for (int c0 = 0; c0 < p.BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tcol + c0, v);
-        tmem_wait_ld();
-        if constexpr (kGluRows) {
-          // Even rows hold gate values, odd rows the up values of the same feature.
-          const int fcol = tl.ft * 64 + (fr >> 1);
-          const bool is_gate = (lane & 1) == 0;
+      const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c0 = 0; c0 < p.BN; c0 += 16) {
+        float v[16];
+        {
+          // Issue the loads of every partial accumulator, then wait once.
+          uint32_t u0[16], u1[16], u2[16];
+          tmem_ld_32x32b_x16(tcol + c0, u0);
+          if (nacc > 1) tmem_ld_32x32b_x16(tcol + static_cast<uint32_t>(p.acc_cols) + c0, u1);
+          if (nacc > 2) tmem_ld_32x32b_x16(tcol + static_cast<uint32_t>(2 * p.acc_cols) + c0, u2);
+          tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float mine = __uint_as_float(v[j]);
-            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-            const int c = c0 + j;
-            const int row = tl.row0 + c;
-            if (c < p.BN && row < tl.row_end) {
-              const int64_t r64 = static_cast<int64_t>(row);
-              if (is_gate) {
-                p.out[r64 * p.ldo + fcol] = __float2bfloat16_rn(silu_f(mine) * other);
-                if (p.saved) p.saved[r64 * N + fcol] = __float2bfloat16_rn(mine);
-              } else if (p.saved) {
-                p.saved[r64 * N + N / 2 + fcol] = __float2bfloat16_rn(mine);
-              }
+          for (int jj = 0; jj < 16; ++jj) {
+            float x = __uint_as_float(u0[jj]);
+            if (nacc > 1) x += __uint_as_float(u1[jj]);
+            if (nacc > 2) x += __uint_as_float(u2[jj]);
+            v[jj] = x;
+          }
+        }
+        const int nrows = min(16, min(p.BN - c0, tl.row_end - (tl.row0 + c0)));
+        if constexpr (kGluRows) {
+          // Lanes 0-15 hold gate values, lanes 16-31 the up values of the same
+          // 16 features. Staging row (64 BF16): [0,16) h, [16,32) g, [32,48) u.
+          const int pr = lane & 15;
+          const bool is_gate = lane < 16;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[jj], 16);
+            uint16_t* row = stg_ptr + jj * 64;
+            if (is_gate) {
+              row[pr] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_f(v[jj]) * other));
+              row[16 + pr] = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
+            } else {
+              row[32 + pr] = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
             }
           }
+          __syncwarp();
+          // 16 H features of this warp: 32 B per row = 2 chunks; g and u likewise.
+          const int fcol = tl.ft * 64 + q * 16;
+          const int nseg = p.saved ? 3 : 1;
+          for (int idx = lane; idx < 16 * 2 * nseg; idx += 32) {
+            const int seg = idx / 32, rr = (idx % 32) >> 1, ch = idx & 1;
+            if (rr < nrows) {
+              const uint4 val = *reinterpret_cast<const uint4*>(stg_ptr + rr * 64 + seg * 16 + ch * 8);
+              const int64_t grow = static_cast<int64_t>(tl.row0 + c0 + rr);
+              __nv_bfloat16* dst = (seg == 0) ? p.out + grow * p.ldo + fcol
+                                 : (seg == 1) ? p.saved + grow * N + fcol
+                                              : p.saved + grow * N + N / 2 + fcol;
+              *reinterpret_cast<uint4*>(dst + ch * 8) = val;
+            }
+          }
+          __syncwarp();
         } else if constexpr (MODE == kModeBwd && EPI == MOE_EPI_SWIGLU_BWD) {
           const int f = tl.ft * kTileF + fr;      // feature of dh (< K)
-          if (f < p.F) {
+          // Staging row: [0,32) dg, [32,64) du of this warp's 32 features.
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = c0 + j;
-              const int row = tl.row0 + c;
-              if (c < p.BN && row < tl.row_end) {
-                const int64_t rb = static_cast<int64_t>(row) * (2 * K);
-                const float g = __bfloat162float(p.saved[rb + f]);
-                const float u = __bfloat162float(p.saved[rb + K + f]);
-                const float dh = __uint_as_float(v[j]);
-                const float s = 1.0f / (1.0f + expf(-g));
-                p.out[rb + f] = __float2bfloat16_rn(dh * u * s * (1.0f + g * (1.0f - s)));
-                p.out[rb + K + f] = __float2bfloat16_rn(dh * g * s);
+          for (int jj = 0; jj < 16; ++jj) {
+            uint16_t dg = 0, du = 0;
+            if (jj < nrows && f < p.F) {
+              const int64_t rb = static_cast<int64_t>(tl.row0 + c0 + jj) * (2 * K);
+              const float g = __bfloat162float(p.saved[rb + f]);
+              const float u = __bfloat162float(p.saved[rb + K + f]);
+              const float s = 1.0f / (1.0f + expf(-g));
+              dg = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj] * u * s * (1.0f + g * (1.0f - s))));
+              du = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj] * g * s));
+            }
+            stg_ptr[jj * 64 + lane] = dg;
+            stg_ptr[jj * 64 + 32 + lane] = du;
+          }
+          __syncwarp();
+          const int fb = tl.ft * kTileF + q * 32;
+          if (fb < p.F) {
+            for (int idx = lane; idx < 16 * 8; idx += 32) {
+              const int rr = idx >> 3, ch = idx & 7;     // 8 chunks: 4 of dg, 4 of du
+              if (rr < nrows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(stg_ptr + rr * 64 + ch * 8);
+                const int64_t rb = static_cast<int64_t>(tl.row0 + c0 + rr) * (2 * K);
+                __nv_bfloat16* dst = p.out + rb + (ch < 4 ? 0 : K) + fb + (ch & 3) * 8;
+                *reinterpret_cast<uint4*>(dst) = val;
               }
             }
           }
+          __syncwarp();
         } else {
-          const int f = tl.ft * kTileF + fr;
-          if (f < p.F) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int c = c0 + j;
-              const int row = tl.row0 + c;
-              if (c < p.BN && row < tl.row_end)
-                p.out[static_cast<int64_t>(row) * p.ldo + f] =
-                    __float2bfloat16_rn(__uint_as_float(v[j]));
+          for (int jj = 0; jj < 16; ++jj)
+            stg_ptr[jj * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
+          __syncwarp();
+          const int fb = tl.ft * kTileF + q * 32;
+          if (fb < p.F) {
+            for (int idx = lane; idx < 16 * 4; idx += 32) {
+              const int rr = idx >> 2, ch = idx & 3;
+              if (rr < nrows) {
+                const uint4 val = *reinterpret_cast<const uint4*>(stg_ptr + rr * 32 + ch * 8);
+                *reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(tl.row0 + c0 + rr) * p.ldo +
+                                          fb + ch * 8) = val;
+              }
             }
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty(buf));
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
 
@@ -500,15 +639,21 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& 
   return cudaErrorInvalidValue;
 }
 
-uint32_t gemm_stage_bytes(int BN, int fmt) {
-  const uint32_t sc = 256u * (fmt == MOE_W_INT4_G32_BF16 ? 2u : 1u);
-  const uint32_t b = kABytes + static_cast<uint32_t>(BN) * 128u + kWqBytes + sc;
+uint32_t gemm_stage_bytes(int mode, int BN, int fmt) {
+  const uint32_t el = (fmt == MOE_W_INT4_G32_BF16) ? 2u : 1u;
+  uint32_t b;
+  if (mode == kModeFwd)   // B 2 chunks, packed 128 rows x 64 B, scales 4 x 128
+    b = static_cast<uint32_t>(BN) * 256u + 8192u + 512u * el;
+  else                    // B 1 chunk, A 16 KiB, packed 64 rows x 64 B, scales 4 x 64
+    b = static_cast<uint32_t>(BN) * 128u + kABytes + 4096u + 256u * el;
   return (b + 1023u) & ~1023u;
 }
 
-uint32_t gemm_fixed_smem_bytes(int stages, int E) {
-  // barriers, TMEM slot + abort flag (16 B), warp totals, tile list, alignment slack
-  return 8u * (3u * stages + 5u) + 16u + 32u * 4u + static_cast<uint32_t>(E + 1) * 4u + 1024u;
+uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E) {
+  // barriers, TMEM slot + abort flag (16 B), warp totals, tile list, epilogue
+  // staging (4 x 4 KiB, 128-byte aligned), alignment slack
+  return 8u * (2u * stages + 2u * a_stages + 3u) + 16u + 32u * 4u +
+         static_cast<uint32_t>(E + 1) * 4u + 128u + 4u * 4096u + 1024u;
 }
 
 }  // namespace moeq

@@ -19,11 +19,13 @@ struct GemmArgs {
   int32_t M;                  // rows of a / dout / out
   int32_t BN;                 // token rows per tile (multiple of 16, <= 256)
   int32_t n_ftiles;           // feature tiles per expert
-  int32_t acc_cols;           // TMEM columns per accumulator buffer (>= BN, multiple of 32)
+  int32_t n_issuers;          // MMA-issuing warps (1..3), each with a partial accumulator
+  int32_t acc_cols;           // TMEM columns per partial accumulator (>= BN, multiple of 32)
   int32_t tmem_cols;          // TMEM columns allocated (power of two, >= 2 * acc_cols)
   int32_t F;                  // output features (fwd: N or N/2 with SwiGLU; bwd: K)
   int32_t R;                  // reduction length (fwd: K; bwd: N)
-  int32_t stages;             // pipeline depth
+  int32_t stages;             // shared-memory fills in flight
+  int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages)
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
   __nv_bfloat16* out;         // [M][ldo]
   int64_t ldo;
@@ -33,8 +35,11 @@ struct GemmArgs {
 cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& tb,
                                  const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
                                  int grid, size_t smem, cudaStream_t s);
-uint32_t gemm_stage_bytes(int BN, int fmt);
-uint32_t gemm_fixed_smem_bytes(int stages, int E);
-constexpr int kGemmThreads = 384;
+uint32_t gemm_stage_bytes(int mode, int BN, int fmt);
+uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E);
+// Warp roles: TMA producer, MMA issuer, two spare warps, kDqGroups dequant
+// warpgroups, one epilogue warpgroup.
+constexpr int kDqGroups = 3;
+constexpr int kGemmThreads = 32 * (4 + 4 * kDqGroups + 4);
 
 }  // namespace moeq

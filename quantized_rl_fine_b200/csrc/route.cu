@@ -5,19 +5,20 @@
 // activates the experts its router selects, and the selected experts are
 // batched into fixed-size groups before the grouped GEMM.
 //
-// Three kernels, no host round trip:
-//  1. route_topk_kernel: one warp per token (8 tokens per warp, 64 per
-//     block); k rounds of a warp-wide argmax (ties to the lower expert id),
-//     softmax of the k selected logits, and a per-block expert histogram in
-//     shared memory.
+// Four kernels, no host round trip:
+//  1. route_topk_kernel: one warp per token (2 tokens per warp, 64 per
+//     1024-thread block); k rounds of a warp-wide argmax (ties to the lower
+//     expert id), softmax of the k selected logits, and a per-block expert
+//     histogram in shared memory.
 //  2. route_scan_kernel: one block; per expert, an exclusive scan of the
 //     block histograms (block bases for step 3), then scans over experts for
 //     the offsets, the active list and the chunk table.
 //  3. route_scatter_kernel: per block, a 64-bit token mask per expert built
 //     with shared-memory atomicOr; the rank of token t inside expert e is the
 //     popcount of the mask below t, which gives the stable position
-//     offsets[e] + block_base[e] + rank. The same block copies the token rows
-//     to their permuted positions with 16-byte loads and stores.
+//     offsets[e] + block_base[e] + rank.
+//  4. permute_rows_kernel: one warp per permuted row copies its token row
+//     with 16-byte loads and stores across the whole grid.
 #include "common.cuh"
 #include "launchers.cuh"
 
@@ -27,12 +28,13 @@ namespace {
 
 constexpr int kRouteTokensPerBlock = 64;
 constexpr int kRouteThreads = 256;
+constexpr int kTopkThreads = 1024;
 
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kTopkThreads)
 route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                   int32_t* __restrict__ topk_idx, float* __restrict__ gates,
                   int32_t* __restrict__ block_counts) {
@@ -40,7 +42,7 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per_warp = kRouteTokensPerBlock / (kRouteThreads / 32);
+  const int per_warp = kRouteTokensPerBlock / (kTopkThreads / 32);
   const int nper = (E + 31) / 32;     // logits per lane (<= 32)
   for (int u = 0; u < per_warp; ++u) {
     const int t = blockIdx.x * kRouteTokensPerBlock + warp * per_warp + u;
@@ -168,12 +170,10 @@ route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk
 __global__ void __launch_bounds__(kRouteThreads)
 route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ block_base,
                      const int32_t* __restrict__ offsets, int T, int E, int k,
-                     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm,
-                     const uint4* __restrict__ x, uint4* __restrict__ x_perm, int64_t row_vec) {
-  extern __shared__ uint32_t sm[];      // lo[E], hi[E], pos[64 * k]
+                     int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
+  extern __shared__ uint32_t sm[];      // lo[E], hi[E]
   uint32_t* lo = sm;
   uint32_t* hi = sm + E;
-  int32_t* pos = reinterpret_cast<int32_t*>(sm + 2 * E);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     lo[e] = 0;
     hi[e] = 0;
@@ -197,16 +197,27 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
     const int p = offsets[e] + base[e] + rank;
     perm_token[p] = t0 + tl;
     inv_perm[static_cast<int64_t>(t0) * k + i] = p;
-    pos[i] = p;
   }
-  if (x == nullptr) return;
-  __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = warp; i < nent; i += kRouteThreads / 32) {
-    const uint4* src = x + static_cast<int64_t>(t0 + i / k) * row_vec;
-    uint4* dst = x_perm + static_cast<int64_t>(pos[i]) * row_vec;
-    for (int64_t c = lane; c < row_vec; c += 32) dst[c] = src[c];
+}
+
+// One warp per permuted row p: x_perm[p] = x[perm_token[p]] (16-byte moves).
+__global__ void __launch_bounds__(256)
+permute_rows_kernel(const int32_t* __restrict__ perm_token, int M, const uint4* __restrict__ x,
+                    uint4* __restrict__ x_perm, int64_t row_vec) {
+  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (p >= M) return;
+  const uint4* src = x + static_cast<int64_t>(perm_token[p]) * row_vec;
+  uint4* dst = x_perm + static_cast<int64_t>(p) * row_vec;
+  int64_t c = lane;
+  for (; c + 96 < row_vec; c += 128) {
+    const uint4 a0 = src[c], a1 = src[c + 32], a2 = src[c + 64], a3 = src[c + 96];
+    dst[c] = a0;
+    dst[c + 32] = a1;
+    dst[c + 64] = a2;
+    dst[c + 96] = a3;
   }
+  for (; c < row_vec; c += 32) dst[c] = src[c];
 }
 
 }  // namespace
@@ -221,7 +232,7 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                          int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
                          void* x_perm, int32_t* block_counts, cudaStream_t s) {
   const int nblk = route_num_blocks(T);
-  route_topk_kernel<<<nblk, kRouteThreads, E * sizeof(int32_t), s>>>(logits, T, E, k, topk_idx,
+  route_topk_kernel<<<nblk, kTopkThreads, E * sizeof(int32_t), s>>>(logits, T, E, k, topk_idx,
                                                                      gates, block_counts);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -229,10 +240,14 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                                        num_active, chunk_offsets, num_chunks);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const size_t sm = (2 * E + kRouteTokensPerBlock * k) * sizeof(uint32_t);
-  route_scatter_kernel<<<nblk, kRouteThreads, sm, s>>>(
-      topk_idx, block_counts, offsets, T, E, k, perm_token, inv_perm,
-      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), d / 8);
+  const size_t sm = 2 * E * sizeof(uint32_t);
+  route_scatter_kernel<<<nblk, kRouteThreads, sm, s>>>(topk_idx, block_counts, offsets, T, E, k,
+                                                       perm_token, inv_perm);
+  err = cudaGetLastError();
+  if (err != cudaSuccess || x == nullptr) return err;
+  const int M = T * k;
+  permute_rows_kernel<<<(M + 7) / 8, 256, 0, s>>>(perm_token, M, static_cast<const uint4*>(x),
+                                                  static_cast<uint4*>(x_perm), d / 8);
   return cudaGetLastError();
 }
 
