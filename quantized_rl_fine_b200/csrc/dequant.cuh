@@ -18,10 +18,20 @@
 
 namespace moeq {
 
+// Each step is written as one explicit PTX instruction: left to the compiler,
+// masks followed by multiplies get rewritten into longer shift/add sequences
+// once the known-zero bits are visible, roughly doubling the instruction count.
+
 // Selector of prmt(w, w >> 4, sel): output bytes {w.byte[p], -, (w>>4).byte[p], -};
 // the high byte of each half is masked away afterwards.
 __device__ __forceinline__ uint32_t pair_select(int p) {
   return static_cast<uint32_t>(p | (p << 4) | ((4 + p) << 8) | ((4 + p) << 12));
+}
+
+// Selector of prmt(lo, hi, sel): output bytes {lo.byte[p], 0, hi.byte[p], 0}. The
+// zero bytes use prmt's sign-replicate mode on a byte whose top bit is clear.
+__device__ __forceinline__ uint32_t pair_select_zero(int p) {
+  return static_cast<uint32_t>(p | (0x8 << 4) | ((4 + p) << 8) | (0x8 << 12));
 }
 
 // w >> 4 as a multiply-high, so the shift runs on the FMA pipe and leaves the
@@ -32,14 +42,44 @@ __device__ __forceinline__ uint32_t shr4(uint32_t w) {
   return r;
 }
 
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {  // (a & b) ^ c
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t and_b32(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("and.b32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t mul_lo(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.lo.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub_rn(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul_rn(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // 8 INT4 codes of one 32-bit word -> 4 BF16 pairs, scale pair s2 = {s, s}.
 __device__ __forceinline__ void dequant8_int4(uint32_t w, uint32_t s2, uint32_t (&o)[4]) {
   const uint32_t odd = shr4(w);
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    uint32_t t = prmt(w, odd, pair_select(p));
-    t = (t & 0x000F000Fu) ^ 0x43084308u;           // {136 + q_even, 136 + q_odd}
-    o[p] = bf16x2_mul(bf16x2_sub(t, 0x43084308u), s2);  // (v - 136) * s
+    // {136 + q_even, 136 + q_odd}, then (v - 136) * s
+    const uint32_t t = and_xor(prmt(w, odd, pair_select(p)), 0x000F000Fu, 0x43084308u);
+    o[p] = bf16x2_mul_rn(bf16x2_sub_rn(t, 0x43084308u), s2);
   }
 }
 
@@ -69,15 +109,17 @@ __device__ __forceinline__ MxScale mx_scale(uint32_t X) {
 // multiply (exponents above 128).
 template <bool TWO>
 __device__ __forceinline__ void dequant8_mxfp4(uint32_t w, const MxScale& s, uint32_t (&o)[4]) {
-  const uint32_t odd = shr4(w);
+  const uint32_t lo = and_b32(w, 0x0F0F0F0Fu);          // even codes, one per byte
+  const uint32_t hi = and_b32(shr4(w), 0x0F0F0F0Fu);    // odd codes
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    const uint32_t t = prmt(w, odd, pair_select(p)) & 0x000F000Fu;   // {c_even, c_odd}
-    // c * 0x1040 = (c << 6) + (c << 12): magnitude to bits 8..6, sign to bit 15
-    // (bits 28..31 for the upper half); the mask drops the spare copies.
-    const uint32_t v = (t * 0x1040u) & 0x81C081C0u;
-    uint32_t r = bf16x2_mul(v, s.a);
-    if constexpr (TWO) r = bf16x2_mul(r, s.b);
+    const uint32_t t = prmt(lo, hi, pair_select_zero(p));   // {c_even, 0, c_odd, 0}
+    // c * 0x1040 = (c << 6) + (c << 12) without carries: magnitude to bits
+    // 8..6, sign to bit 15 (bits 24..22 and 31 for the upper half); the mask
+    // drops the spare copies.
+    const uint32_t v = and_b32(mul_lo(t, 0x1040u), 0x81C081C0u);
+    uint32_t r = bf16x2_mul_rn(v, s.a);
+    if constexpr (TWO) r = bf16x2_mul_rn(r, s.b);
     o[p] = r;
   }
 }
