@@ -100,7 +100,7 @@ int choose_bn(int64_t M, int E, int max_bn) {
     if (v >= 16 && v <= max_bn && v % 16 == 0) return v;
   }
   const double mean = static_cast<double>(M) / std::max(1, E);
-  const double want = std::max(1.0, 1.4 * mean);
+  const double want = std::max(1.0, 1.25 * mean);
   const int tiles = static_cast<int>((want + max_bn - 1.0) / max_bn);
   int bn = static_cast<int>((want / tiles + 15.0) / 16.0) * 16;
   return std::min(max_bn, std::max(16, bn));
@@ -140,33 +140,64 @@ struct GemmPlan {
 // Tensor memory (512 columns) holds n_issuers partial accumulators of
 // acc_cols columns each and, in the forward kernels, the A stages (64
 // columns per 128-wide fill). Forward token tiles are capped at 160 rows so
-// that at least four A stages fit; backward tiles (A in shared memory) go up
-// to 256.
+// that one partial and four A stages always fit; backward tiles (A in shared
+// memory) go up to 256.
 GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
   GemmPlan pl;
   pl.BN = choose_bn(M, w->E, mode == kModeFwd ? 160 : 256);
   pl.acc_cols = (pl.BN + 31) / 32 * 32;
   pl.stage_bytes = gemm_stage_bytes(mode, pl.BN, fmt);
-  if (mode == kModeFwd) {
-    // A stage of a 128-wide fill: 64 columns; keep at least four of them.
-    pl.n_issuers = std::max(1, std::min(3, (512 - 4 * 64) / pl.acc_cols));
-    pl.a_stages = std::min(8, (512 - pl.n_issuers * pl.acc_cols) / 64);
-    pl.tmem_cols = 512;
-  } else {
-    pl.n_issuers = std::max(1, std::min(3, 512 / pl.acc_cols));
-    pl.tmem_cols = next_pow2(pl.n_issuers * pl.acc_cols);
+  // MOEQ_NI caps the number of MMA-issuing warps (tuning only).
+  int ni_max = kMaxIssuers;
+  if (const char* env = getenv("MOEQ_NI")) {
+    const int v = atoi(env);
+    if (v >= 1 && v <= kMaxIssuers) ni_max = v;
   }
+  // Every ring has a multiple of kLanes stages, and of n_issuers where the
+  // issuers wait on it (the A ring), so that each stage has one waiter per role.
+  auto ring_step = [](int ni) {
+    int a = kLanes, b = ni;
+    while (b) { const int t = a % b; a = b; b = t; }
+    return kLanes / a * ni;
+  };
   // As many shared-memory fills as fit (at most 16): a deep ring hides the
   // latency of the weight stream.
   const int avail = max_smem_optin();
-  int stages = 16;
-  auto fits = [&](int s) {
-    const int sa = (mode == kModeFwd) ? pl.a_stages : s;
+  auto fits = [&](int s, int sa) {
     return static_cast<int>(s * pl.stage_bytes + gemm_fixed_smem_bytes(s, sa, w->E)) <= avail;
   };
-  while (stages > 4 && !fits(stages)) --stages;
-  pl.stages = stages;
-  if (mode != kModeFwd) pl.a_stages = stages;
+  if (mode == kModeFwd) {
+    // A stage of a 128-wide fill: 64 tensor-memory columns. The most issuers
+    // that still leave two A stages per lane (one issuer always does, as
+    // BN <= 160).
+    pl.n_issuers = 1;
+    pl.a_stages = 2 * kLanes;
+    for (int ni = ni_max; ni >= 1; --ni) {
+      const int step = ring_step(ni);
+      const int room = (512 - ni * pl.acc_cols) / 64;
+      const int sa = std::min(8, room / step * step);
+      if (sa >= 2 * kLanes) {
+        pl.n_issuers = ni;
+        pl.a_stages = sa;
+        break;
+      }
+    }
+    pl.tmem_cols = 512;
+    int stages = 8 * kLanes;
+    while (stages > kLanes && !fits(stages, pl.a_stages)) stages -= kLanes;
+    pl.stages = stages;
+  } else {
+    int stages = 8 * kLanes;
+    while (stages > kLanes && !fits(stages, stages)) stages -= kLanes;
+    pl.stages = stages;
+    pl.a_stages = stages;
+    pl.n_issuers = 1;
+    for (int ni = ni_max; ni >= 1; --ni) {
+      if (ni * pl.acc_cols <= 512 && stages % ring_step(ni) == 0) { pl.n_issuers = ni; break; }
+    }
+    pl.tmem_cols = next_pow2(pl.n_issuers * pl.acc_cols);
+  }
+  const int stages = pl.stages;
   pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
   pl.n_ftiles = (F + tile_f - 1) / tile_f;
   const int64_t bound = static_cast<int64_t>(pl.n_ftiles) *

@@ -35,9 +35,8 @@ namespace moeq {
 namespace {
 
 constexpr int kThreads = kGemmThreads;
-constexpr int kDqWarp0 = 4;                              // first dequant warp
-constexpr int kEpiWarp0 = kDqWarp0 + 4 * kDqGroups;      // first epilogue warp
-static_assert(kThreads == 32 * (kEpiWarp0 + 4), "warp roles must fill the CTA");
+// 24 warps: six on each of the four SM sub-partitions, so 80 registers a thread.
+static_assert(kThreads <= 1024 && ((kThreads / 32 + 3) / 4) * 32 * 80 <= 16384, "roles must fit 80 registers a thread");
 constexpr int kTileF = 128;            // output features per tile (MMA M)
 constexpr uint32_t kABytes = kTileF * 64 * 2;   // 16 KiB dequantized A tile (backward fill)
 
@@ -219,7 +218,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       mbar_init(empty(s), 1);
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(full_a(s), 4);
+      mbar_init(full_a(s), kDqWarpsPerLane);
       mbar_init(a_free(s), 1);
     }
     mbar_init(acc_full, p.n_issuers);
@@ -228,12 +227,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp < kProdWarps && lane == 0) {
     tma_prefetch_desc(&tm_b);
     tma_prefetch_desc(&tm_wq);
     tma_prefetch_desc(&tm_sc);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+  if (warp == kIssuerWarp0) tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -247,92 +246,81 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const int NI = p.n_issuers;
   const uint32_t a_col0 = static_cast<uint32_t>(NI * p.acc_cols);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    // Lanes 0-2 issue the fill's three bulk tensor copies in one instruction:
-    // lane 0 the token rows, lane 1 the packed weights, lane 2 the group scales.
-    if (lane < 3) {
-      const uint64_t policy = (lane == 0) ? l2_policy_evict_last() : l2_policy_evict_first();
-      const CUtensorMap* map = (lane == 0) ? &tm_b : (lane == 1) ? &tm_wq : &tm_sc;
+  if (warp < kProdWarps) {
+    // ------------------------------------------------------------ TMA producers
+    // Producer pw issues fills f with f % kProdWarps == pw: one thread issues
+    // the fill's three bulk tensor copies (token rows, packed weights, group
+    // scales) on the fill's stage f % S. A single thread needs a few hundred
+    // cycles per fill for the barrier wait and the copy issue; two producers
+    // overlap that latency.
+    if (lane == 0) {
+      const int pw = warp;
+      const uint64_t pol_b = l2_policy_evict_last();
+      const uint64_t pol_w = l2_policy_evict_first();
       const uint32_t tx = b_bytes + kWqFill + kScFill;
-      int st = 0;
+      int st = pw;                           // stage of the next own fill
       uint32_t ph = 0;
-      long long fills = 0;
+      long long f0 = 0, last_own = -1;       // first fill of the tile
+      int r0 = 0;                            // f0 % kLanes
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(p, tile_start, A, t);
-        for (int kb = 0; kb < nkb; ++kb) {
-          // Lane 0 waits; the three lanes leave or go on together.
-          int got = 1;
-          if (lane == 0) got = mbar_wait(empty(st), ph ^ 1u, abort_flag) ? 1 : 0;
-          got = __shfl_sync(0x7u, got, 0);
-          if (!got) { ok = false; break; }
-          if (lane == 0) mbar_arrive_expect_tx(full_tma(st), tx);
-          uint32_t dst;
-          int c0, c1, c2;
-          if (lane == 0) {                       // rows x [kFillK] BF16
-            dst = B_at(st);
-            c0 = 0;
-            c1 = tl.row0;
-            c2 = kb * kBChunks;
-          } else if constexpr (MODE == kModeFwd) {
-            if (lane == 1) {                     // packed: [2 halves or 1][rows][64 B]
-              dst = W_at(st);
-              c0 = kb * 64;
-              if constexpr (EPI == MOE_EPI_SWIGLU) { c1 = tl.ft * 64; c2 = 2 * tl.e; }
-              else { c1 = tl.e * N + tl.ft * kTileF; c2 = 0; }
-            } else {                             // scales: [4 groups][128 rows]
-              dst = S_at(st);
-              if constexpr (EPI == MOE_EPI_SWIGLU) { c0 = tl.ft * 64; c1 = 0; c2 = tl.e * (K / 32) + kb * 4; }
-              else { c0 = tl.ft * kTileF; c1 = tl.e * (K / 32) + kb * 4; c2 = 0; }
+        for (int kb = (pw - r0 + kLanes) % kLanes; kb < nkb; kb += kLanes) {
+          const long long f = f0 + kb;
+          if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t bar = full_tma(st);
+          mbar_arrive_expect_tx(bar, tx);
+          tma_load_3d_hint(B_at(st), &tm_b, bar, 0, tl.row0, kb * kBChunks, pol_b);
+          if constexpr (MODE == kModeFwd) {
+            if constexpr (EPI == MOE_EPI_SWIGLU) {
+              // packed: [2 halves][64 rows][64 B]; scales: [4 groups][2 halves][64]
+              tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * 64, tl.ft * 64, 2 * tl.e, pol_w);
+              tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * 64, 0, tl.e * (K / 32) + kb * 4, pol_w);
+            } else {
+              // packed: [128 rows][64 B]; scales: [4 groups][128 rows]
+              tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * 64, tl.e * N + tl.ft * kTileF, 0, pol_w);
+              tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * kTileF, tl.e * (K / 32) + kb * 4, 0, pol_w);
             }
           } else {
-            if (lane == 1) {                     // packed: [64 rows][64 B]
-              dst = W_at(st);
-              c0 = tl.ft * 64;
-              c1 = tl.e * N + kb * kFillK;
-              c2 = 0;
-            } else {                             // scales: [4 groups][64 rows]
-              dst = S_at(st);
-              c0 = kb * kFillK;
-              c1 = tl.e * (K / 32) + tl.ft * 4;
-              c2 = 0;
-            }
+            // packed: [64 rows][64 B]; scales: [4 groups][64 rows]
+            tma_load_3d_hint(W_at(st), &tm_wq, bar, tl.ft * 64, tl.e * N + kb * kFillK, 0, pol_w);
+            tma_load_3d_hint(S_at(st), &tm_sc, bar, kb * kFillK, tl.e * (K / 32) + tl.ft * 4, 0, pol_w);
           }
-          __syncwarp(0x7u);
-          tma_load_3d_hint(dst, map, full_tma(st), c0, c1, c2, policy);
-          ++fills;
-          if (++st == S) { st = 0; ph ^= 1u; }
+          last_own = f;
+          st += kLanes;
+          if (st >= S) { st -= S; ph ^= 1u; }
         }
+        f0 += nkb;
+        r0 = (r0 + nkb) % kLanes;
       }
-      if (!ok && lane == 0) {
-        // Let every issued copy land before the CTA can exit.
-        const long long first = fills > S ? fills - S : 0;
-        for (long long f = first; f < fills; ++f)
-          mbar_drain(full_tma(static_cast<int>(f % S)), static_cast<uint32_t>((f / S) & 1));
+      if (!ok) {
+        // Let this producer's copies that may still be in flight land before
+        // the CTA can exit (its fills within the last S).
+        for (long long g = last_own; g >= 0 && g > last_own - S; g -= kLanes)
+          mbar_drain(full_tma(static_cast<int>(g % S)), static_cast<uint32_t>((g / S) & 1));
       }
     }
-  } else if (warp >= 1 && warp <= NI) {
+  } else if (warp >= kIssuerWarp0 && warp < kIssuerWarp0 + NI) {
     // ------------------------------------------------------------ MMA issuers
     // One thread issuing tcgen05.mma sustains only about one instruction per
-    // ~100 cycles whatever N is, so the K loop of a tile is split among NI
-    // issuing warps: issuer j takes the fills kb with kb % NI == j into its own
-    // partial accumulator; the epilogue adds the partials in a fixed order.
+    // ~100 cycles whatever N is, so the reduction of a tile is split among NI
+    // issuing warps: issuer j takes the fills f with f % NI == j into its own
+    // partial accumulator; the epilogue adds the partials in issuer order.
     if (lane == 0) {
-      const int j = warp - 1;
+      const int j = warp - kIssuerWarp0;
       const uint32_t idesc = idesc_bf16_f32(kTileF, p.BN, MODE == kModeBwd ? 1u : 0u, 0u);
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(j * p.acc_cols);
-      int st = 0, sa = 0;
-      uint32_t ph = 0, pha = 0;
+      int st = j, sa = j;                     // stages of the next own fill (f = j, j + NI, ...)
+      uint32_t pha = 0;
       int it = 0;
+      int r0 = 0;                             // (first fill of the tile) % NI
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
         if (!mbar_wait(acc_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint32_t acc = 0;
-        int r = 0;                            // kb % NI
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (r == j) {
+        for (int kb = (j - r0 + NI) % NI; kb < nkb; kb += NI) {
+          {
             if (!mbar_wait(full_a(sa), pha, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
@@ -359,20 +347,26 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             mma_commit(empty(st));
             if constexpr (kTmemA) mma_commit(a_free(sa));
           }
-          if (++r == NI) r = 0;
-          if (++st == S) { st = 0; ph ^= 1u; }
-          if (++sa == SA) { sa = 0; pha ^= 1u; }
+          st += NI;
+          if (st >= S) st -= S;
+          sa += NI;
+          if (sa >= SA) { sa -= SA; pha ^= 1u; }
         }
+        r0 = (r0 + nkb) % NI;
         if (ok) mma_commit(acc_full);         // arrives even when this issuer had no fill
       }
       // All MMAs of this CTA done before tensor memory is released.
       mma_commit(drain_bar);
       mbar_drain(drain_bar, 0);
     }
-  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + 4 * kDqGroups) {
+  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kLanes * kDqWarpsPerLane) {
     // ------------------------------------------------------------ dequantizers
-    // kDqGroups warpgroups take the fills in turn (fill f goes to group f % kDqGroups).
-    const int grp = (warp - kDqWarp0) >> 2;
+    // kLanes groups of kDqWarpsPerLane warps take the fills in turn (fill f
+    // goes to group f % kLanes). In a group, warp (q, hk) covers tensor-memory
+    // lane quarter q and half hk of the fill's 128 reduction elements.
+    static_assert(kDqWarpsPerLane == 8, "two warps per lane quarter");
+    const int grp = (warp - kDqWarp0) / kDqWarpsPerLane;
+    const int hk = ((warp - kDqWarp0) >> 2) & 1;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int i = q * 32 + lane;            // A row (forward) / thread slot (backward)
     // Forward: A row i is one output feature. With SwiGLU each warp's 32 rows
@@ -381,23 +375,22 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     // phase of a 128-bit shared load touches 8 distinct swizzle slots.
     const int src = kGluRows ? ((lane < 16) ? (16 * q + lane) : (64 + 16 * q + lane - 16)) : i;
     // Fill f of the CTA uses stage f % S with parity (f / S) & 1; this group
-    // owns fills grp, grp + kDqGroups, ... and steps its stage and parity
-    // incrementally (kDqGroups < S).
-    int turn = 0;                           // f % kDqGroups
+    // owns fills grp, grp + kLanes, ... and steps its stage and parity
+    // incrementally.
+    int r0 = 0;                             // (first fill of the tile) % kLanes
     int st = grp, sa = grp;                 // fill ring and A ring positions of the next own fill
     uint32_t ph = 0, pha = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const bool mine = (turn == grp);
-        if (++turn == kDqGroups) turn = 0;
-        if (!mine) continue;
+      const int kb_first = (grp - r0 + kLanes) % kLanes;
+      r0 = (r0 + nkb) % kLanes;
+      for (int kb = kb_first; kb < nkb; kb += kLanes) {
         const int cur = st, cur_a = sa;
         const uint32_t cur_ph = ph, cur_pha = pha;
         const int kb_cur = kb;
-        st += kDqGroups;
+        st += kLanes;
         if (st >= S) { st -= S; ph ^= 1u; }
-        sa += kDqGroups;
+        sa += kLanes;
         if (sa >= SA) { sa -= SA; pha ^= 1u; }
         if (!mbar_wait(full_tma(cur), cur_ph, abort_flag)) { ok = false; break; }
         // Forward: the A stage must have been released by the MMAs of the
@@ -410,44 +403,42 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           // index ^= (row >> 1) & 3). Scales: [4 groups][128 rows].
           const uint32_t prow = wq + src * 64;
           const uint32_t sw = (src >> 1) & 3;
+          const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a_col0 +
+                                static_cast<uint32_t>(cur_a * 64);
+          // The two 32-element groups of this warp's half; each is stored to
+          // tensor memory as soon as it is dequantized (16 columns, two BF16
+          // per column, low half = even k), which keeps only 16 results live.
+          // A half past the reduction length (K % 128 == 64) is written as
+          // zeros, so neither the zero-filled codes nor a foreign scale can
+          // reach the MMA.
+          const bool zero_half = kb_cur * kFillK + hk * 64 >= p.R;
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            uint32_t o[32];
-            // A half fill past the reduction length (K % 128 == 64) is zero, so
-            // neither the zero-filled codes nor a foreign scale can reach the MMA.
-            if (kb_cur * kFillK + h2 * 64 >= p.R) {
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * hk + cc;
+            uint32_t o[16];
+            if (zero_half) {
 #pragma unroll
-              for (int jj = 0; jj < 32; ++jj) o[jj] = 0u;
+              for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
             } else {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int c = 2 * h2 + h;     // 32-element group of this fill
               const uint4 pk = lds128(prow + ((c ^ sw) << 4));
               const uint32_t soff = c * 128 + src;
               const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
                                                                   : lds_u8(sc + soff);
-              uint32_t oh[16];
-              dequant32<FMT>(pk, sbits, oh);
-#pragma unroll
-              for (int jj = 0; jj < 16; ++jj) o[16 * h + jj] = oh[jj];
+              dequant32<FMT>(pk, sbits, o);
             }
-            }
-            // Lane i of the A sub-stage: 32 columns = 64 BF16 along K, low half = even k.
-            tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a_col0 +
-                                   static_cast<uint32_t>(cur_a * 64 + h2 * 32),
-                               o);
+            tmem_st_32x32b_x16(trow + static_cast<uint32_t>(c * 16), o);
           }
           tmem_wait_st();
           tc_fence_before();
         } else {
-          // Thread = (reduction row r, feature half hf): 64 features = 2 groups.
-          // Packed rows are 64 bytes with the TMA 64-byte swizzle (chunk ^= (r >> 1) & 3).
-          // Scales: [4 groups][64 rows].
+          // Thread = (reduction row r, feature half hf, group jh = hk of that
+          // half): 32 features. Packed rows are 64 bytes with the TMA 64-byte
+          // swizzle (chunk ^= (r >> 1) & 3). Scales: [4 groups][64 rows].
           const uint32_t a_st = A_at(cur);
           const int r = i & 63;
           const int hf = i >> 6;
-#pragma unroll
-          for (int jh = 0; jh < 2; ++jh) {
+          {
+            const int jh = hk;
             const int c = 2 * hf + jh;
             const uint4 pk = lds128(wq + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
             const uint32_t soff = c * 64 + r;
@@ -479,28 +470,45 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     const int fr = q * 32 + lane;           // accumulator row = tile feature
     const uint32_t stg = stg_base + static_cast<uint32_t>(q) * 4096u;
     uint16_t* stg_ptr = reinterpret_cast<uint16_t*>(gbase + (stg - base));
-    const int nacc = NI < nkb ? NI : nkb;
+    static_assert(kMaxIssuers <= 3, "the epilogue sums at most three partial accumulators");
     int it = 0;
+    int r0 = 0;                             // (first fill of the tile) % NI
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const Tile tl = decode_tile(p, tile_start, A, t);
+      // Issuer j wrote its partial in this tile iff one of the tile's nkb
+      // fills f has f % NI == j.
+      const bool has0 = ((NI - r0) % NI) < nkb;
+      const bool has1 = NI > 1 && ((1 + NI - r0) % NI) < nkb;
+      const bool has2 = NI > 2 && ((2 + NI - r0) % NI) < nkb;
+      r0 = (r0 + nkb) % NI;
+      // Tensor-memory column offsets of the written partials, in issuer order.
+      const uint32_t acc = static_cast<uint32_t>(p.acc_cols);
+      const int nv = int(has0) + int(has1) + int(has2);
+      const uint32_t pc0 = has0 ? 0u : (has1 ? acc : 2 * acc);
+      const uint32_t pc1 = (has0 && has1) ? acc : 2 * acc;
+      const uint32_t pc2 = 2 * acc;
       if (!mbar_wait(acc_full, static_cast<uint32_t>(it & 1), abort_flag)) break;
       tc_fence_after();
       const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < p.BN; c0 += 16) {
         float v[16];
         {
-          // Issue the loads of every partial accumulator, then wait once.
-          uint32_t u0[16], u1[16], u2[16];
-          tmem_ld_32x32b_x16(tcol + c0, u0);
-          if (nacc > 1) tmem_ld_32x32b_x16(tcol + static_cast<uint32_t>(p.acc_cols) + c0, u1);
-          if (nacc > 2) tmem_ld_32x32b_x16(tcol + static_cast<uint32_t>(2 * p.acc_cols) + c0, u2);
+          // The partials written in this tile, in issuer order: the first two
+          // loaded together, the third after them.
+          uint32_t ua[16], ub[16];
+          tmem_ld_32x32b_x16(tcol + pc0 + c0, ua);
+          if (nv > 1) tmem_ld_32x32b_x16(tcol + pc1 + c0, ub);
           tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
-            float x = __uint_as_float(u0[jj]);
-            if (nacc > 1) x += __uint_as_float(u1[jj]);
-            if (nacc > 2) x += __uint_as_float(u2[jj]);
-            v[jj] = x;
+            v[jj] = __uint_as_float(ua[jj]);
+            if (nv > 1) v[jj] += __uint_as_float(ub[jj]);
+          }
+          if (nv > 2) {
+            tmem_ld_32x32b_x16(tcol + pc2 + c0, ua);
+            tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) v[jj] += __uint_as_float(ua[jj]);
           }
         }
         const int nrows = min(16, min(p.BN - c0, tl.row_end - (tl.row0 + c0)));
@@ -595,7 +603,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, p.tmem_cols);
+  if (warp == kIssuerWarp0) tmem_dealloc(tmem_base, p.tmem_cols);
 }
 
 }  // namespace

@@ -19,13 +19,14 @@ struct GemmArgs {
   int32_t M;                  // rows of a / dout / out
   int32_t BN;                 // token rows per tile (multiple of 16, <= 256)
   int32_t n_ftiles;           // feature tiles per expert
-  int32_t n_issuers;          // MMA-issuing warps (1..3), each with a partial accumulator
+  int32_t n_issuers;          // MMA-issuing warps (1..kMaxIssuers), each with a partial accumulator
   int32_t acc_cols;           // TMEM columns per partial accumulator (>= BN, multiple of 32)
   int32_t tmem_cols;          // TMEM columns allocated (power of two, >= 2 * acc_cols)
   int32_t F;                  // output features (fwd: N or N/2 with SwiGLU; bwd: K)
   int32_t R;                  // reduction length (fwd: K; bwd: N)
-  int32_t stages;             // shared-memory fills in flight
-  int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages)
+  int32_t stages;             // shared-memory fills in flight (multiple of kLanes and n_issuers)
+  int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages);
+                              // multiple of kLanes and n_issuers
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
   __nv_bfloat16* out;         // [M][ldo]
   int64_t ldo;
@@ -37,9 +38,23 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& 
                                  int grid, size_t smem, cudaStream_t s);
 uint32_t gemm_stage_bytes(int mode, int BN, int fmt);
 uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E);
-// Warp roles: TMA producer, MMA issuer, two spare warps, kDqGroups dequant
-// warpgroups, one epilogue warpgroup.
-constexpr int kDqGroups = 3;
-constexpr int kGemmThreads = 32 * (4 + 4 * kDqGroups + 4);
+// Warp roles, in order: kLanes TMA producers, up to kLanes MMA-issuing warps,
+// kLanes dequant groups of kDqWarpsPerLane warps (two per tensor-memory lane
+// quarter, one per half of the fill's reduction span), one epilogue
+// warpgroup. Fill f (the CTA's f-th 128-wide reduction step, counted across
+// tiles) belongs to pipeline lane f % kLanes: its producer, its dequant group
+// and (with kLanes issuers) its MMA issuer. The shared-memory ring and the
+// tensor-memory A ring have a multiple of kLanes stages, so each stage is
+// waited on by exactly one member of each role, which sees every phase of the
+// stage's barriers: a phase-parity wait can then never mistake a phase two
+// behind for the one it waits for.
+constexpr int kLanes = 2;
+constexpr int kDqWarpsPerLane = 8;
+constexpr int kProdWarps = kLanes;
+constexpr int kMaxIssuers = kLanes;
+constexpr int kIssuerWarp0 = kProdWarps;
+constexpr int kDqWarp0 = kIssuerWarp0 + kMaxIssuers;
+constexpr int kEpiWarp0 = kDqWarp0 + kLanes * kDqWarpsPerLane;
+constexpr int kGemmThreads = 32 * (kEpiWarp0 + 4);
 
 }  // namespace moeq
