@@ -11,18 +11,23 @@
 // One persistent CTA per SM walks a device-built tile list (active experts in
 // ascending id, which is chunk order; inside an expert, feature tile major and
 // token tile minor). A tile is 128 output features x BN token rows (BN a
-// multiple of 16, <= 256), accumulated in FP32 in tensor memory by
-// tcgen05.mma with the dequantized weight as operand A (M = 128) and the
-// token rows as operand B (N = BN):
+// multiple of 16), accumulated in FP32 in tensor memory by tcgen05.mma with
+// the dequantized weight as operand A (M = 128) and the token rows as operand
+// B (N = BN):
 //
-//   forward  D[f, t] = sum_k W[e][f][k] * a[t][k]     (A K-major)
-//   backward D[f, t] = sum_n W[e][n][f] * dout[t][n]  (A MN-major)
+//   forward  D[f, t] = sum_k W[e][f][k] * a[t][k]     (A K-major, in tensor memory)
+//   backward D[f, t] = sum_n W[e][n][f] * dout[t][n]  (A MN-major, in shared memory)
 //
-// Warp roles (384 threads): warp 0 lane 0 issues TMA loads (token rows,
-// packed weights, group scales) into a ring of stages; warp 1 owns tensor
-// memory and lane 0 issues the MMAs; warps 4-7 dequantize each stage into a
-// 128B-swizzled BF16 tile; warps 8-11 drain the double-buffered accumulator
-// (epilogue: plain, SwiGLU, SwiGLU backward) while the next tile runs.
+// The reduction is walked in fills of 128 (forward) or 64 (backward)
+// elements. Fill f of the CTA belongs to pipeline lane f % kLanes, which has
+// its own TMA producer warp (token rows, packed weights and group scales into
+// a shared-memory stage), its own dequant group (eight warps: packed codes to
+// BF16 in registers, then into the A stage) and, with kLanes issuers, its own
+// MMA-issuing warp that accumulates its fills into a partial accumulator. One
+// issuing thread sustains only about one tcgen05.mma per ~100+ cycles, so
+// splitting the reduction across issuers is what keeps the tensor core fed at
+// small N. An epilogue warpgroup sums the partials in issuer order and writes
+// BF16 (plain, SwiGLU with the saved gate/up, or the SwiGLU backward).
 // Every wait is bounded; on a timeout the kernel records a device error,
 // lets its in-flight copies and MMAs finish (again bounded), frees tensor
 // memory and returns.

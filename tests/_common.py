@@ -58,3 +58,35 @@ def assert_close_intermediate(got: np.ndarray, want: np.ndarray, what: str, abs_
     lim = abs_tol + bf16_ulp(want)
     bad = err > lim
     assert not np.any(bad), f"{what}: {int(bad.sum())} elements out of tolerance, worst {float(err.max()):.3e}"
+
+
+def adapter_grad_bound(x_rows: np.ndarray, dxa_rows: np.ndarray, row_expert: np.ndarray, E: int,
+                       base: float = 2e-2) -> np.ndarray:
+    """Element bound for the FP32 adapter gradient dR[e,b,i,j] = sum_p x[p,32b+i] dx'[p,32b+j].
+
+    dx' is a BF16 intermediate: the library and the oracle may round each of
+    its elements to neighbouring BF16 values (their FP32 sums differ in
+    order), so dR may differ by up to sum_p |x[p,32b+i]| * ulp(dx'[p,32b+j]),
+    plus the base absolute tolerance of the final outputs.
+    """
+    nb = x_rows.shape[1] // 32
+    out = np.zeros((E, nb, 32, 32))
+    ax = np.abs(x_rows).reshape(x_rows.shape[0], nb, 32)
+    ul = bf16_ulp(dxa_rows).reshape(dxa_rows.shape[0], nb, 32)
+    for e in range(E):
+        sel = row_expert == e
+        out[e] = np.einsum("mbi,mbj->bij", ax[sel], ul[sel])
+    return base + out
+
+
+def assert_close_bounded(got: np.ndarray, want: np.ndarray, bound: np.ndarray, what: str,
+                         rel_l2: float = REL_L2):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape == bound.shape, (what, got.shape, want.shape, bound.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    err = np.abs(got - want)
+    bad = err > bound
+    rl2 = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30))
+    assert not np.any(bad) and rl2 <= rel_l2, \
+        f"{what}: {int(bad.sum())} elements above their bound, rel-L2 {rl2:.3e}"
