@@ -34,6 +34,9 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
+// NPER: logits held per lane (>= ceil(E / 32)); the selection loops run over
+// exactly NPER slots.
+template <int NPER>
 __global__ void __launch_bounds__(kTopkThreads)
 route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                   int32_t* __restrict__ topk_idx, float* __restrict__ gates,
@@ -43,16 +46,15 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per_warp = kRouteTokensPerBlock / (kTopkThreads / 32);
-  const int nper = (E + 31) / 32;     // logits per lane (<= 32)
   for (int u = 0; u < per_warp; ++u) {
     const int t = blockIdx.x * kRouteTokensPerBlock + warp * per_warp + u;
     if (t >= T) break;
     const float* row = logits + static_cast<int64_t>(t) * E;
-    float v[32];
+    float v[NPER];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < NPER; ++i) {
       const int e = lane + 32 * i;
-      v[i] = (i < nper && e < E) ? row[e] : 0.0f;
+      v[i] = (e < E) ? row[e] : 0.0f;
     }
     uint32_t taken = 0;
     float my_val = 0.0f;
@@ -61,9 +63,9 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
       float bv = -INFINITY;
       int bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < NPER; ++i) {
         const int e = lane + 32 * i;
-        if (i < nper && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
+        if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) {
           bv = v[i];
           bi = e;
         }
@@ -232,8 +234,19 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                          int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
                          void* x_perm, int32_t* block_counts, cudaStream_t s) {
   const int nblk = route_num_blocks(T);
-  route_topk_kernel<<<nblk, kTopkThreads, E * sizeof(int32_t), s>>>(logits, T, E, k, topk_idx,
-                                                                     gates, block_counts);
+  const int nper = (E + 31) / 32;
+  const size_t hsm = E * sizeof(int32_t);
+#define MOEQ_TOPK(N_)                                                                         \
+  route_topk_kernel<N_><<<nblk, kTopkThreads, hsm, s>>>(logits, T, E, k, topk_idx, gates,     \
+                                                        block_counts)
+  if (nper <= 1) MOEQ_TOPK(1);
+  else if (nper <= 2) MOEQ_TOPK(2);
+  else if (nper <= 4) MOEQ_TOPK(4);
+  else if (nper <= 8) MOEQ_TOPK(8);
+  else if (nper <= 12) MOEQ_TOPK(12);
+  else if (nper <= 16) MOEQ_TOPK(16);
+  else MOEQ_TOPK(32);
+#undef MOEQ_TOPK
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, chunk_size, offsets, active,
