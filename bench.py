@@ -61,7 +61,11 @@ def _workloads():
         "train_int4": C.TRAIN_INT4,
     }
     for T in C.TRILLION_T_SWEEP:
-        w[f"trillion_int4_T{T}"] = C.TRILLION_INT4.with_(T=T)
+        w[f"trillion_int4_T{T}"] = C.TRILLION_INT4.with_(T=T, name=f"{C.TRILLION_INT4.name}_T{T}")
+    # The per-expert shape of the decode step (about 2.7 token rows per active
+    # expert) with 48 experts: small enough for a full ncu capture.
+    w["trillion_int4_E48_T16"] = C.TRILLION_INT4.with_(
+        E=48, T=16, name="trillion_int4_E48_k8_d7168_f2048_T16")
     return w
 
 
@@ -415,8 +419,19 @@ def run_ours(args, cfg):
         graphs.append(g)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    for i in range(args.warmup):
+    # Training with several ranks: the shared adapter's gradient is summed over
+    # the ranks after every step (the path's only collective), eagerly after
+    # the graph replay so every rank issues the same collectives in order.
+    from quantized_rl_fine_b200 import dp as dp_mod
+    reduce_grad = cfg.train and cfg.adapter and world > 1
+
+    def run_step(i):
         graphs[i % ROTATE].replay()
+        if reduce_grad:
+            dp_mod.allreduce_adapter_grad(keep[i % ROTATE]["d_adapter"])
+
+    for i in range(args.warmup):
+        run_step(i)
     torch.cuda.synchronize()
 
     # ---------------------------------------------------------------- timed region
@@ -427,7 +442,7 @@ def run_ours(args, cfg):
     with ClockSampler(local) as clocks:
         t0.record(stream)
         for i in range(args.steps):
-            graphs[i % ROTATE].replay()
+            run_step(i)
         t1.record(stream)
         torch.cuda.synchronize()
     if world > 1:
@@ -487,7 +502,7 @@ def run_ours(args, cfg):
         wl["logits"].copy_(hl, non_blocking=True)
         if hy is not None:
             wl["dy"].copy_(hy, non_blocking=True)
-        graphs[i % ROTATE].replay()
+        run_step(i)
         hout[i % ROTATE].copy_(keep[i % ROTATE][out_key], non_blocking=True)
     for i in range(max(3, args.warmup)):
         e2e_step(i)
