@@ -296,6 +296,15 @@ def _cpu_baseline(cfg, budget_s=20.0):
                        f"{flops / 1e9:.2f} GFLOP in {secs:.2f} s")
 
 
+def _config_dict(cfg, chunk, world):
+    """The workload description both arms print."""
+    return {"workload": cfg.name, "E": cfg.E, "k": cfg.k, "d": cfg.d, "f": cfg.f,
+            "T_per_gpu": cfg.T, "fmt": cfg.fmt, "chunk_size": chunk,
+            "adapter": cfg.adapter, "train": cfg.train,
+            "l2": f"{ROTATE} rotating input sets, larger than L2 together",
+            "parallelism": f"dp{world} (replicated weights, own tokens per GPU)"}
+
+
 def run_reference(args, cfg):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -316,8 +325,7 @@ def run_reference(args, cfg):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "E": cfg.E, "k": cfg.k, "d": cfg.d, "f": cfg.f,
-                   "T": cfg.T, "fmt": cfg.fmt},
+        "config": _config_dict(cfg, args.chunk or cfg.chunk_size, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(),
                          "kind": "oracle",
                          "sample": f"each step: routing of all {cfg.T} tokens + the GEMMs of "
@@ -553,11 +561,7 @@ def run_ours(args, cfg):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "E": cfg.E, "k": cfg.k, "d": cfg.d, "f": cfg.f,
-                   "T_per_gpu": cfg.T, "fmt": cfg.fmt, "chunk_size": chunk,
-                   "adapter": cfg.adapter, "train": cfg.train,
-                   "l2": f"{ROTATE} rotating input sets, larger than L2 together",
-                   "parallelism": f"dp{world} (replicated weights, own tokens per GPU)"},
+        "config": _config_dict(cfg, chunk, world),
         "weight_gbs": world * acc["wbytes"] / (ms_per_step * 1e-3) / 1e9,
         "roofline": roof,
         "e2e": {"value": world * step_flops / (e_ms / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
