@@ -100,7 +100,7 @@ int choose_bn(int64_t M, int E, int max_bn) {
     if (v >= 16 && v <= max_bn && v % 16 == 0) return v;
   }
   const double mean = static_cast<double>(M) / std::max(1, E);
-  const double want = std::max(1.0, 1.25 * mean);
+  const double want = std::max(1.0, 1.5 * mean);
   const int tiles = static_cast<int>((want + max_bn - 1.0) / max_bn);
   int bn = static_cast<int>((want / tiles + 15.0) / 16.0) * 16;
   return std::min(max_bn, std::max(16, bn));
@@ -139,12 +139,13 @@ struct GemmPlan {
 // SwiGLU forward, whose tile holds 64 gate and the 64 matching up rows).
 // Tensor memory (512 columns) holds n_issuers partial accumulators of
 // acc_cols columns each and, in the forward kernels, the A stages (64
-// columns per 128-wide fill). Forward token tiles are capped at 160 rows so
-// that one partial and four A stages always fit; backward tiles (A in shared
-// memory) go up to 256.
+// columns per 128-wide fill). Forward token tiles are capped at 96 rows: two
+// partials and four A stages fit, and the token-row box leaves room for six
+// shared-memory stages (wider tiles measured slower for want of ring depth);
+// backward tiles (A in shared memory) go up to 256.
 GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
   GemmPlan pl;
-  pl.BN = choose_bn(M, w->E, mode == kModeFwd ? 160 : 256);
+  pl.BN = choose_bn(M, w->E, mode == kModeFwd ? 96 : 256);
   pl.acc_cols = (pl.BN + 31) / 32 * 32;
   pl.stage_bytes = gemm_stage_bytes(mode, pl.BN, fmt);
   // MOEQ_NI caps the number of MMA-issuing warps (tuning only).
@@ -169,7 +170,7 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   if (mode == kModeFwd) {
     // A stage of a 128-wide fill: 64 tensor-memory columns. The most issuers
     // that still leave two A stages per lane (one issuer always does, as
-    // BN <= 160).
+    // BN <= 96).
     pl.n_issuers = 1;
     pl.a_stages = 2 * kLanes;
     for (int ni = ni_max; ni >= 1; --ni) {

@@ -86,10 +86,13 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
 
 struct Tile {
   int e, ft, row0, row_end;
+  int width;  // token rows of the tile's MMA (multiple of 16, <= BN)
 };
 
 // Tile t of the tile list: active index a with tile_start[a] <= t (shared
-// memory), then feature tile major, token tile minor inside the expert.
+// memory), then feature tile major, token tile minor inside the expert. An
+// expert's m rows are split into nrt = ceil(m / BN) token tiles of equal width
+// (ceil(m / nrt) rounded up to 16), so the MMAs run on few padding rows.
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* tile_start, int A,
                                             int t) {
   int lo = 0, hi = A - 1;
@@ -102,10 +105,12 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* ti
   const int local = t - tile_start[lo];
   const int seg0 = p.offsets[r.e];
   const int seg1 = p.offsets[r.e + 1];
-  const int nrt = (seg1 - seg0 + p.BN - 1) / p.BN;
+  const int m = seg1 - seg0;
+  const int nrt = (m + p.BN - 1) / p.BN;
+  r.width = (((m + nrt - 1) / nrt) + 15) & ~15;
   r.ft = local / nrt;
-  r.row0 = seg0 + (local - r.ft * nrt) * p.BN;
-  r.row_end = seg1;
+  r.row0 = seg0 + (local - r.ft * nrt) * r.width;
+  r.row_end = min(seg1, r.row0 + r.width);
   return r;
 }
 
@@ -162,7 +167,12 @@ __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* 
   return A;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+// SiLU and the logistic function with the fast exponential and division
+// intrinsics (a few fp32 ulps): their results are rounded to BF16 right after,
+// and the epilogue runs them for every output element while the dequant warps
+// compete for the same issue slots.
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int MODE, int FMT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -313,7 +323,6 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     // partial accumulator; the epilogue adds the partials in issuer order.
     if (lane == 0) {
       const int j = warp - kIssuerWarp0;
-      const uint32_t idesc = idesc_bf16_f32(kTileF, p.BN, MODE == kModeBwd ? 1u : 0u, 0u);
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(j * p.acc_cols);
       int st = j, sa = j;                     // stages of the next own fill (f = j, j + NI, ...)
       uint32_t pha = 0;
@@ -321,6 +330,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       int r0 = 0;                             // (first fill of the tile) % NI
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const uint32_t idesc = idesc_bf16_f32(kTileF, decode_tile(p, tile_start, A, t).width,
+                                              MODE == kModeBwd ? 1u : 0u, 0u);
         if (!mbar_wait(acc_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint32_t acc = 0;
@@ -495,7 +506,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       if (!mbar_wait(acc_full, static_cast<uint32_t>(it & 1), abort_flag)) break;
       tc_fence_after();
       const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      for (int c0 = 0; c0 < p.BN; c0 += 16) {
+      for (int c0 = 0; c0 < tl.width; c0 += 16) {
         float v[16];
         {
           // The partials written in this tile, in issuer order: the first two
@@ -516,7 +527,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             for (int jj = 0; jj < 16; ++jj) v[jj] += __uint_as_float(ua[jj]);
           }
         }
-        const int nrows = min(16, min(p.BN - c0, tl.row_end - (tl.row0 + c0)));
+        const int nrows = min(16, tl.row_end - (tl.row0 + c0));
         if constexpr (kGluRows) {
           // Lanes 0-15 hold gate values, lanes 16-31 the up values of the same
           // 16 features. Staging row (64 BF16): [0,16) h, [16,32) g, [32,48) u.
@@ -559,7 +570,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
               const int64_t rb = static_cast<int64_t>(tl.row0 + c0 + jj) * (2 * K);
               const float g = __bfloat162float(p.saved[rb + f]);
               const float u = __bfloat162float(p.saved[rb + K + f]);
-              const float s = 1.0f / (1.0f + expf(-g));
+              const float s = sigmoid_f(g);
               dg = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj] * u * s * (1.0f + g * (1.0f - s))));
               du = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj] * g * s));
             }
