@@ -139,13 +139,12 @@ struct GemmPlan {
 // SwiGLU forward, whose tile holds 64 gate and the 64 matching up rows).
 // Tensor memory (512 columns) holds n_issuers partial accumulators of
 // acc_cols columns each and, in the forward kernels, the A stages (64
-// columns per 128-wide fill). Forward token tiles are capped at 96 rows: two
-// partials and four A stages fit, and the token-row box leaves room for six
-// shared-memory stages (wider tiles measured slower for want of ring depth);
-// backward tiles (A in shared memory) go up to 256.
+// columns per 128-wide fill). Token tiles are capped at 96 rows: two partials
+// and four A stages fit, and the token-row box leaves room for six
+// shared-memory stages (wider tiles measured slower, forward and backward).
 GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
   GemmPlan pl;
-  pl.BN = choose_bn(M, w->E, mode == kModeFwd ? 96 : 256);
+  pl.BN = choose_bn(M, w->E, 96);
   pl.acc_cols = (pl.BN + 31) / 32 * 32;
   pl.stage_bytes = gemm_stage_bytes(mode, pl.BN, fmt);
   // MOEQ_NI caps the number of MMA-issuing warps (tuning only).
