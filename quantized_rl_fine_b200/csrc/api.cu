@@ -130,7 +130,7 @@ moe_status check_groups(const moe_groups* g, int E) {
 }
 
 struct GemmPlan {
-  int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers;
+  int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers, lanes;
   uint32_t stage_bytes;
   size_t smem;
 };
@@ -153,12 +153,22 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
     const int v = atoi(env);
     if (v >= 1 && v <= kMaxIssuers) ni_max = v;
   }
-  // Every ring has a multiple of kLanes stages, and of n_issuers where the
-  // issuers wait on it (the A ring), so that each stage has one waiter per role.
-  auto ring_step = [](int ni) {
-    int a = kLanes, b = ni;
+  // Pipeline lanes: four (one dequant warp per lane quarter, 128 elements per
+  // thread and fill) while a token tile of at most 64 rows leaves room for a
+  // ring of eight or more stages; two (two warps per quarter) for wider tiles,
+  // whose stages would otherwise be too few. MOEQ_LANES overrides (tuning).
+  pl.lanes = pl.BN <= 64 ? 4 : 2;
+  if (const char* env = getenv("MOEQ_LANES")) {
+    const int v = atoi(env);
+    if (v == 2 || v == 4) pl.lanes = v;
+  }
+  const int L = pl.lanes;
+  // Every ring has a multiple of L stages, and of n_issuers where the issuers
+  // wait on it (the A ring), so that each stage has one waiter per role.
+  auto ring_step = [L](int ni) {
+    int a = L, b = ni;
     while (b) { const int t = a % b; a = b; b = t; }
-    return kLanes / a * ni;
+    return L / a * ni;
   };
   // As many shared-memory fills as fit (at most 16): a deep ring hides the
   // latency of the weight stream.
@@ -168,27 +178,26 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   };
   if (mode == kModeFwd) {
     // A stage of a 128-wide fill: 64 tensor-memory columns. The most issuers
-    // that still leave two A stages per lane (one issuer always does, as
-    // BN <= 96).
+    // that still leave four A stages (one issuer always does, as BN <= 96).
     pl.n_issuers = 1;
-    pl.a_stages = 2 * kLanes;
+    pl.a_stages = 4;
     for (int ni = ni_max; ni >= 1; --ni) {
       const int step = ring_step(ni);
       const int room = (512 - ni * pl.acc_cols) / 64;
       const int sa = std::min(8, room / step * step);
-      if (sa >= 2 * kLanes) {
+      if (sa >= 4) {
         pl.n_issuers = ni;
         pl.a_stages = sa;
         break;
       }
     }
     pl.tmem_cols = 512;
-    int stages = 8 * kLanes;
-    while (stages > kLanes && !fits(stages, pl.a_stages)) stages -= kLanes;
+    int stages = 16;
+    while (stages > L && !fits(stages, pl.a_stages)) stages -= L;
     pl.stages = stages;
   } else {
-    int stages = 8 * kLanes;
-    while (stages > kLanes && !fits(stages, stages)) stages -= kLanes;
+    int stages = 16;
+    while (stages > L && !fits(stages, stages)) stages -= L;
     pl.stages = stages;
     pl.a_stages = stages;
     pl.n_issuers = 1;
@@ -302,7 +311,7 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ldo = ldo;
   p.saved = static_cast<__nv_bfloat16*>(saved);
-  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, tb, tw, ts, p, pl.grid, pl.smem, s));
+  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, pl.lanes, tb, tw, ts, p, pl.grid, pl.smem, s));
 }
 
 }  // namespace

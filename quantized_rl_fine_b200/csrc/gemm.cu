@@ -19,14 +19,14 @@
 //   backward D[f, t] = sum_n W[e][n][f] * dout[t][n]  (A MN-major, in shared memory)
 //
 // The reduction is walked in fills of 128 (forward) or 64 (backward)
-// elements. Fill f of the CTA belongs to pipeline lane f % kLanes, which has
-// its own TMA producer warp (token rows, packed weights and group scales into
-// a shared-memory stage), its own dequant group (eight warps: packed codes to
-// BF16 in registers, then into the A stage) and, with kLanes issuers, its own
-// MMA-issuing warp that accumulates its fills into a partial accumulator. One
-// issuing thread sustains only about one tcgen05.mma per ~100+ cycles, so
-// splitting the reduction across issuers is what keeps the tensor core fed at
-// small N. An epilogue warpgroup sums the partials in issuer order and writes
+// elements. Fill f of the CTA belongs to pipeline lane f % kLanes, whose
+// dequant group (four warps, one per tensor-memory lane quarter) turns its
+// packed codes into BF16 in registers and then into the A stage; producer
+// warp f % kProdWarps issues its copies (token rows, packed weights, group
+// scales) into a shared-memory stage, and MMA-issuing warp f % n_issuers
+// accumulates it into that issuer's partial accumulator. One issuing thread
+// sustains only about one tcgen05.mma per 70-150 cycles, so splitting the
+// reduction across issuers is what keeps the tensor core fed at small N. An epilogue warpgroup sums the partials in issuer order and writes
 // BF16 (plain, SwiGLU with the saved gate/up, or the SwiGLU backward).
 // Every wait is bounded; on a timeout the kernel records a device error,
 // lets its in-flight copies and MMAs finish (again bounded), frees tensor
@@ -174,11 +174,16 @@ __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* 
 __device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int MODE, int FMT, int EPI>
+template <int MODE, int FMT, int EPI, int LANES>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_wq,
                      const __grid_constant__ CUtensorMap tm_sc, const GemmArgs p) {
+  constexpr int kLanes = LANES;
+  constexpr int kDqWarpsPerLane = kDqWarps / LANES;   // 4 or 8
+  constexpr int kParts = kDqWarpsPerLane / 4;         // warps per lane quarter
+  static_assert(LANES % kProdWarps == 0 && LANES % kMaxIssuers == 0, "lanes own their stages");
+  static_assert(kDqWarpsPerLane % 4 == 0 && (kParts == 1 || kParts == 2), "whole lane quarters");
   constexpr uint32_t kScEl = (FMT == MOE_W_INT4_G32_BF16) ? 2 : 1;
   constexpr bool kGluRows = (MODE == kModeFwd && EPI == MOE_EPI_SWIGLU);
   // Forward: fills of 128 reduction elements; the dequantized A tile goes to
@@ -276,11 +281,11 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       int st = pw;                           // stage of the next own fill
       uint32_t ph = 0;
       long long f0 = 0, last_own = -1;       // first fill of the tile
-      int r0 = 0;                            // f0 % kLanes
+      int r0 = 0;                            // f0 % kProdWarps
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile(p, tile_start, A, t);
-        for (int kb = (pw - r0 + kLanes) % kLanes; kb < nkb; kb += kLanes) {
+        for (int kb = (pw - r0 + kProdWarps) % kProdWarps; kb < nkb; kb += kProdWarps) {
           const long long f = f0 + kb;
           if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t bar = full_tma(st);
@@ -302,16 +307,16 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             tma_load_3d_hint(S_at(st), &tm_sc, bar, kb * kFillK, tl.e * (K / 32) + tl.ft * 4, 0, pol_w);
           }
           last_own = f;
-          st += kLanes;
+          st += kProdWarps;
           if (st >= S) { st -= S; ph ^= 1u; }
         }
         f0 += nkb;
-        r0 = (r0 + nkb) % kLanes;
+        r0 = (r0 + nkb) % kProdWarps;
       }
       if (!ok) {
         // Let this producer's copies that may still be in flight land before
         // the CTA can exit (its fills within the last S).
-        for (long long g = last_own; g >= 0 && g > last_own - S; g -= kLanes)
+        for (long long g = last_own; g >= 0 && g > last_own - S; g -= kProdWarps)
           mbar_drain(full_tma(static_cast<int>(g % S)), static_cast<uint32_t>((g / S) & 1));
       }
     }
@@ -379,10 +384,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     // ------------------------------------------------------------ dequantizers
     // kLanes groups of kDqWarpsPerLane warps take the fills in turn (fill f
     // goes to group f % kLanes). In a group, warp (q, hk) covers tensor-memory
-    // lane quarter q and half hk of the fill's 128 reduction elements.
-    static_assert(kDqWarpsPerLane == 8, "two warps per lane quarter");
+    // lane quarter q (32 rows of the A tile) and part hk of the kParts parts
+    // of the fill's reduction span (forward: 4 / kParts 32-element groups).
     const int grp = (warp - kDqWarp0) / kDqWarpsPerLane;
-    const int hk = ((warp - kDqWarp0) >> 2) & 1;
+    const int hk = ((warp - kDqWarp0) >> 2) % kParts;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int i = q * 32 + lane;            // A row (forward) / thread slot (backward)
     // Forward: A row i is one output feature. With SwiGLU each warp's 32 rows
@@ -421,18 +426,17 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           const uint32_t sw = (src >> 1) & 3;
           const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a_col0 +
                                 static_cast<uint32_t>(cur_a * 64);
-          // The two 32-element groups of this warp's half; each is stored to
-          // tensor memory as soon as it is dequantized (16 columns, two BF16
-          // per column, low half = even k), which keeps only 16 results live.
-          // A half past the reduction length (K % 128 == 64) is written as
-          // zeros, so neither the zero-filled codes nor a foreign scale can
-          // reach the MMA.
-          const bool zero_half = kb_cur * kFillK + hk * 64 >= p.R;
+          // The four 32-element groups of the fill; each is stored to tensor
+          // memory as soon as it is dequantized (16 columns, two BF16 per
+          // column, low half = even k), which keeps only 16 results live. A
+          // half past the reduction length (K % 128 == 64) is written as zeros,
+          // so neither the zero-filled codes nor a foreign scale can reach the
+          // MMA.
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * hk + cc;
+          for (int cc = 0; cc < 4 / kParts; ++cc) {
+            const int c = hk * (4 / kParts) + cc;
             uint32_t o[16];
-            if (zero_half) {
+            if (kb_cur * kFillK + (c >> 1) * 64 >= p.R) {
 #pragma unroll
               for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
             } else {
@@ -447,14 +451,16 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           tmem_wait_st();
           tc_fence_before();
         } else {
-          // Thread = (reduction row r, feature half hf, group jh = hk of that
-          // half): 32 features. Packed rows are 64 bytes with the TMA 64-byte
-          // swizzle (chunk ^= (r >> 1) & 3). Scales: [4 groups][64 rows].
+          // Thread = (reduction row r, feature half hf): 64 features = 2
+          // groups, split over the kParts warps of the lane quarter. Packed
+          // rows are 64 bytes with the TMA 64-byte swizzle (chunk ^= (r >> 1)
+          // & 3). Scales: [4 groups][64 rows].
           const uint32_t a_st = A_at(cur);
           const int r = i & 63;
           const int hf = i >> 6;
-          {
-            const int jh = hk;
+#pragma unroll
+          for (int jj = 0; jj < 2 / kParts; ++jj) {
+            const int jh = hk * (2 / kParts) + jj;
             const int c = 2 * hf + jh;
             const uint4 pk = lds128(wq + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
             const uint32_t soff = c * 64 + r;
@@ -624,11 +630,11 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
 
 }  // namespace
 
-template <int MODE, int FMT, int EPI>
+template <int MODE, int FMT, int EPI, int LANES>
 static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorMap& tw,
                                           const CUtensorMap& ts, const GemmArgs& p, int grid,
                                           size_t smem, cudaStream_t s) {
-  auto k = grouped_qgemm_kernel<MODE, FMT, EPI>;
+  auto k = grouped_qgemm_kernel<MODE, FMT, EPI, LANES>;
   // Raise the dynamic shared-memory limit once per (device, kernel); later
   // calls, including ones under stream capture, skip it.
   static int set_for[64] = {0};
@@ -645,12 +651,14 @@ static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorM
   return cudaGetLastError();
 }
 
-cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& tb,
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, const CUtensorMap& tb,
                                  const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
                                  int grid, size_t smem, cudaStream_t s) {
-#define MOEQ_CASE(M_, F_, E_)                                               \
-  if (mode == M_ && fmt == F_ && epi == E_)                                 \
-    return launch_grouped_qgemm_t<M_, F_, E_>(tb, tw, ts, p, grid, smem, s);
+#define MOEQ_CASE(M_, F_, E_)                                                          \
+  if (mode == M_ && fmt == F_ && epi == E_)                                            \
+    return lanes == 4 ? launch_grouped_qgemm_t<M_, F_, E_, 4>(tb, tw, ts, p, grid, smem, s) \
+                      : launch_grouped_qgemm_t<M_, F_, E_, 2>(tb, tw, ts, p, grid, smem, s);
+  if (lanes != 2 && lanes != 4) return cudaErrorInvalidValue;
   MOEQ_CASE(kModeFwd, MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
   MOEQ_CASE(kModeFwd, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU)
   MOEQ_CASE(kModeFwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)

@@ -24,37 +24,36 @@ struct GemmArgs {
   int32_t tmem_cols;          // TMEM columns allocated (power of two, >= 2 * acc_cols)
   int32_t F;                  // output features (fwd: N or N/2 with SwiGLU; bwd: K)
   int32_t R;                  // reduction length (fwd: K; bwd: N)
-  int32_t stages;             // shared-memory fills in flight (multiple of kLanes and n_issuers)
+  int32_t stages;             // shared-memory fills in flight (multiple of the lane count)
   int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages);
-                              // multiple of kLanes and n_issuers
+                              // multiple of the lane count
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
   __nv_bfloat16* out;         // [M][ldo]
   int64_t ldo;
   __nv_bfloat16* saved;       // fwd SwiGLU: written [M][N]; bwd SwiGLU: read [M][2K]
 };
 
-cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, const CUtensorMap& tb,
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, const CUtensorMap& tb,
                                  const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
                                  int grid, size_t smem, cudaStream_t s);
 uint32_t gemm_stage_bytes(int mode, int BN, int fmt);
 uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E);
-// Warp roles, in order: kLanes TMA producers, up to kLanes MMA-issuing warps,
-// kLanes dequant groups of kDqWarpsPerLane warps (two per tensor-memory lane
-// quarter, one per half of the fill's reduction span), one epilogue
-// warpgroup. Fill f (the CTA's f-th 128-wide reduction step, counted across
-// tiles) belongs to pipeline lane f % kLanes: its producer, its dequant group
-// and (with kLanes issuers) its MMA issuer. The shared-memory ring and the
-// tensor-memory A ring have a multiple of kLanes stages, so each stage is
-// waited on by exactly one member of each role, which sees every phase of the
-// stage's barriers: a phase-parity wait can then never mistake a phase two
-// behind for the one it waits for.
-constexpr int kLanes = 2;
-constexpr int kDqWarpsPerLane = 8;
-constexpr int kProdWarps = kLanes;
-constexpr int kMaxIssuers = kLanes;
+// Warp roles, in order: kProdWarps TMA producers, up to kMaxIssuers
+// MMA-issuing warps, kDqWarps dequant warps split into LANES groups (LANES is a
+// kernel template parameter, 2 or 4), one epilogue warpgroup. Fill f (the
+// CTA's f-th 128-wide reduction step, counted across tiles) belongs to
+// pipeline lane f % LANES (its dequant group), to producer f % kProdWarps and
+// to issuer f % n_issuers. The shared-memory ring and the tensor-memory A ring
+// have a multiple of LANES stages (LANES is a multiple of both other counts),
+// so each stage is waited on by exactly one member of each role, which sees
+// every phase of the stage's barriers: a phase-parity wait can then never
+// mistake a phase two behind for the one it waits for.
+constexpr int kProdWarps = 2;
+constexpr int kMaxIssuers = 2;
+constexpr int kDqWarps = 16;
 constexpr int kIssuerWarp0 = kProdWarps;
 constexpr int kDqWarp0 = kIssuerWarp0 + kMaxIssuers;
-constexpr int kEpiWarp0 = kDqWarp0 + kLanes * kDqWarpsPerLane;
+constexpr int kEpiWarp0 = kDqWarp0 + kDqWarps;
 constexpr int kGemmThreads = 32 * (kEpiWarp0 + 4);
 
 }  // namespace moeq
