@@ -92,17 +92,19 @@ int max_smem_optin() {
   return n;
 }
 
-// Token rows per tile from the mean rows per expert: ~1.4x the mean split
-// into as few tiles of <= max_bn as possible, rounded up to a multiple of 16.
+// Token rows per tile from the mean rows per expert, rounded up to a multiple
+// of 16 and capped at max_bn (MOEQ_BN overrides, tuning only).
 int choose_bn(int64_t M, int E, int max_bn) {
   if (const char* env = getenv("MOEQ_BN")) {
     const int v = atoi(env);
     if (v >= 16 && v <= max_bn && v % 16 == 0) return v;
   }
+  // 1.5x the mean rows per expert, so that most experts fit one token tile
+  // (their weights are streamed once); experts with more rows are split by
+  // the kernel into equal tiles of at most BN rows.
   const double mean = static_cast<double>(M) / std::max(1, E);
   const double want = std::max(1.0, 1.5 * mean);
-  const int tiles = static_cast<int>((want + max_bn - 1.0) / max_bn);
-  int bn = static_cast<int>((want / tiles + 15.0) / 16.0) * 16;
+  const int bn = static_cast<int>((std::min(want, static_cast<double>(max_bn)) + 15.0) / 16.0) * 16;
   return std::min(max_bn, std::max(16, bn));
 }
 
