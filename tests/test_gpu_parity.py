@@ -255,3 +255,18 @@ def test_mxfp4_up_projection_full_size():
 
 def test_device_error_word_is_clear_after_runs():
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+# ----------------------------------------------------------------------------- every kernel variant
+
+@pytest.mark.parametrize("lanes,bn", [(2, 16), (2, 48), (2, 96), (4, 16), (4, 48), (4, 64)])
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, RAGGED_MX], ids=["int4", "mxfp4_ragged"])
+def test_each_lane_count_and_tile_width_matches_the_oracle(monkeypatch, cfg, lanes, bn):
+    """The planner picks one lane count per shape; this runs every pipeline
+    variant (two or four lanes, forward and backward, both formats, with and
+    without the K % 128 == 64 tail) at several token-tile widths on the same
+    inputs and checks each against the oracle."""
+    monkeypatch.setenv("MOEQ_LANES", str(lanes))
+    monkeypatch.setenv("MOEQ_BN", str(bn))
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
