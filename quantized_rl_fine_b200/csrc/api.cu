@@ -133,6 +133,7 @@ moe_status check_groups(const moe_groups* g, int E) {
 
 struct GemmPlan {
   int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers, lanes;
+  bool pair;  // forward on CTA pairs (M = 256 MMAs)
   uint32_t stage_bytes;
   size_t smem;
 };
@@ -146,9 +147,19 @@ struct GemmPlan {
 // shared-memory stages (wider tiles measured slower, forward and backward).
 GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f, int fmt) {
   GemmPlan pl;
-  pl.BN = choose_bn(M, w->E, 96);
+  pl.n_ftiles = (F + tile_f - 1) / tile_f;
+  // CTA pairs (forward, an even number of feature tiles): one M = 256 MMA per
+  // K step of two SMs' weight tiles, and each SM loads half of the token
+  // rows. Opt-in with MOEQ_PAIR=1.
+  pl.pair = false;
+  if (const char* env = getenv("MOEQ_PAIR")) pl.pair = (atoi(env) == 1);
+  pl.pair = pl.pair && mode == kModeFwd && pl.n_ftiles % 2 == 0;
+  // A pair's CTAs hold half of the token rows each, so its tiles may be twice
+  // as wide for the same shared memory per stage.
+  pl.BN = choose_bn(M, w->E, pl.pair ? 192 : 96);
+  if (pl.pair) pl.BN = (pl.BN + 31) / 32 * 32;   // pair MMAs take N in steps of 32
   pl.acc_cols = (pl.BN + 31) / 32 * 32;
-  pl.stage_bytes = gemm_stage_bytes(mode, pl.BN, fmt);
+  pl.stage_bytes = gemm_stage_bytes(mode, pl.BN, fmt, pl.pair);
   // MOEQ_NI caps the number of MMA-issuing warps (tuning only).
   int ni_max = kMaxIssuers;
   if (const char* env = getenv("MOEQ_NI")) {
@@ -210,10 +221,12 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   }
   const int stages = pl.stages;
   pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
-  pl.n_ftiles = (F + tile_f - 1) / tile_f;
-  const int64_t bound = static_cast<int64_t>(pl.n_ftiles) *
+  const int64_t bound = static_cast<int64_t>(pl.pair ? pl.n_ftiles / 2 : pl.n_ftiles) *
                         (std::min<int64_t>(w->E, M) + (M + pl.BN - 1) / pl.BN);
-  pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound)));
+  if (pl.pair)   // CTAs, two per pair tile; the launch clamps to the resident pairs
+    pl.grid = 2 * static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms() / 2, bound)));
+  else
+    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound)));
   return pl;
 }
 
@@ -251,7 +264,7 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   {  // token rows: [M][R] BF16 viewed as (64, M, R/64) -> smem [chunk][BN rows][64]
     const uint64_t dims[3] = {64, static_cast<uint64_t>(M), static_cast<uint64_t>(R) / 64};
     const uint64_t strides[2] = {static_cast<uint64_t>(R) * 2, 128};
-    const uint32_t box[3] = {64, static_cast<uint32_t>(pl.BN), chunks};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(pl.pair ? pl.BN / 2 : pl.BN), chunks};
     if (!make_map_3d(&tb, bmat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return MOE_ERR_CUDA;
@@ -301,7 +314,7 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   p.K = w->K;
   p.M = static_cast<int32_t>(M);
   p.BN = pl.BN;
-  p.n_ftiles = pl.n_ftiles;
+  p.n_ftiles = pl.pair ? pl.n_ftiles / 2 : pl.n_ftiles;
   p.n_issuers = pl.n_issuers;
   p.acc_cols = pl.acc_cols;
   p.tmem_cols = pl.tmem_cols;
@@ -313,7 +326,7 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ldo = ldo;
   p.saved = static_cast<__nv_bfloat16*>(saved);
-  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, pl.lanes, tb, tw, ts, p, pl.grid, pl.smem, s));
+  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, pl.lanes, pl.pair, tb, tw, ts, p, pl.grid, pl.smem, s));
 }
 
 }  // namespace

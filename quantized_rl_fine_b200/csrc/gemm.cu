@@ -31,6 +31,8 @@
 // Every wait is bounded; on a timeout the kernel records a device error,
 // lets its in-flight copies and MMAs finish (again bounded), frees tensor
 // memory and returns.
+#include <algorithm>
+
 #include "common.cuh"
 #include "dequant.cuh"
 #include "gemm.cuh"
@@ -92,7 +94,9 @@ struct Tile {
 // Tile t of the tile list: active index a with tile_start[a] <= t (shared
 // memory), then feature tile major, token tile minor inside the expert. An
 // expert's m rows are split into nrt = ceil(m / BN) token tiles of equal width
-// (ceil(m / nrt) rounded up to 16), so the MMAs run on few padding rows.
+// (ceil(m / nrt) rounded up to kRound, 16, or 32 for CTA-pair MMAs), so the
+// MMAs run on few padding rows.
+template <int kRound>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* tile_start, int A,
                                             int t) {
   int lo = 0, hi = A - 1;
@@ -107,7 +111,7 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* ti
   const int seg1 = p.offsets[r.e + 1];
   const int m = seg1 - seg0;
   const int nrt = (m + p.BN - 1) / p.BN;
-  r.width = (((m + nrt - 1) / nrt) + 15) & ~15;
+  r.width = (((m + nrt - 1) / nrt) + kRound - 1) & ~(kRound - 1);
   r.ft = local / nrt;
   r.row0 = seg0 + (local - r.ft * nrt) * r.width;
   r.row_end = min(seg1, r.row0 + r.width);
@@ -174,7 +178,7 @@ __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* 
 __device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int MODE, int FMT, int EPI, int LANES>
+template <int MODE, int FMT, int EPI, int LANES, int PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_wq,
@@ -184,6 +188,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   constexpr int kParts = kDqWarpsPerLane / 4;         // warps per lane quarter
   static_assert(LANES % kProdWarps == 0 && LANES % kMaxIssuers == 0, "lanes own their stages");
   static_assert(kDqWarpsPerLane % 4 == 0 && (kParts == 1 || kParts == 2), "whole lane quarters");
+  // PAIR: a cluster of two CTAs works on 256 output features (128 each) of
+  // the same token tile with M = 256 MMAs issued by the even CTA; each CTA
+  // loads and dequantizes its own weight rows and loads half of the token
+  // rows (forward only).
+  static_assert(!PAIR || MODE == kModeFwd, "CTA pairs run the forward kernels");
+  constexpr int kWRound = PAIR ? 32 : 16;
   constexpr uint32_t kScEl = (FMT == MOE_W_INT4_G32_BF16) ? 2 : 1;
   constexpr bool kGluRows = (MODE == kModeFwd && EPI == MOE_EPI_SWIGLU);
   // Forward: fills of 128 reduction elements; the dequantized A tile goes to
@@ -203,7 +213,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
 
   const int S = p.stages;
   const uint32_t stage_bytes = p.stage_bytes;
-  const uint32_t b_chunk = static_cast<uint32_t>(p.BN) * 128u;   // one [BN][64] BF16 chunk
+  // One [rows][64] BF16 chunk of token rows; a pair's CTAs hold BN / 2 rows each.
+  const uint32_t b_chunk = static_cast<uint32_t>(PAIR ? p.BN / 2 : p.BN) * 128u;
   const uint32_t b_bytes = b_chunk * kBChunks;
   // One stage: [B kBChunks x BN*128][A 16 KiB (backward only)][packed][scales]
   auto B_at = [&](int s) { return base + s * stage_bytes; };
@@ -231,6 +242,11 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Position in the pair (0 issues the MMAs and owns the barriers they wait
+  // on) and the tile walk: a pair takes tile t, t + pairs, ...
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -238,11 +254,11 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       mbar_init(empty(s), 1);
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(full_a(s), kDqWarpsPerLane);
+      mbar_init(full_a(s), PAIR ? 2 * kDqWarpsPerLane : kDqWarpsPerLane);
       mbar_init(a_free(s), 1);
     }
     mbar_init(acc_full, p.n_issuers);
-    mbar_init(acc_empty, 4);
+    mbar_init(acc_empty, PAIR ? 8 : 4);
     mbar_init(drain_bar, p.n_issuers);
     *abort_flag = 0;
     fence_barrier_init();
@@ -252,14 +268,25 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     tma_prefetch_desc(&tm_wq);
     tma_prefetch_desc(&tm_sc);
   }
-  if (warp == kIssuerWarp0) tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+  if (warp == kIssuerWarp0) {
+    if constexpr (PAIR) tmem_alloc_pair(smem_u32(tmem_slot), p.tmem_cols);
+    else tmem_alloc(smem_u32(tmem_slot), p.tmem_cols);
+  }
   tc_fence_before();
-  __syncthreads();
+  // A pair also waits here until the other CTA's barriers are initialised.
+  if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   const int A = build_tile_list(p, tile_start, warp_tot);
   const int total = tile_start[A];
+  // Tile t of the list as this CTA sees it (a pair's CTAs take feature tiles
+  // 2 ft and 2 ft + 1 of the pair's feature tile ft).
+  auto tile_at = [&](int t) {
+    Tile tl = decode_tile<kWRound>(p, tile_start, A, t);
+    if (PAIR) tl.ft = 2 * tl.ft + static_cast<int>(rank);
+    return tl;
+  };
   const int nkb = (p.R + kFillK - 1) / kFillK;   // forward K % 128 may be 64: zero tail
   const int N = p.N, K = p.K;
   // Tensor-memory columns: [partial accumulator 0 .. NI-1][A stage 0 .. S-1 (forward)].
@@ -283,14 +310,16 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       long long f0 = 0, last_own = -1;       // first fill of the tile
       int r0 = 0;                            // f0 % kProdWarps
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile tl = decode_tile(p, tile_start, A, t);
+      for (int t = t_first; t < total && ok; t += t_step) {
+        const Tile tl = tile_at(t);
+        // A pair's CTAs hold token rows [0, w/2) and [w/2, w) of the tile.
+        const int brow = tl.row0 + static_cast<int>(rank) * (tl.width >> 1);
         for (int kb = (pw - r0 + kProdWarps) % kProdWarps; kb < nkb; kb += kProdWarps) {
           const long long f = f0 + kb;
           if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t bar = full_tma(st);
           mbar_arrive_expect_tx(bar, tx);
-          tma_load_3d_hint(B_at(st), &tm_b, bar, 0, tl.row0, kb * kBChunks, pol_b);
+          tma_load_3d_hint(B_at(st), &tm_b, bar, 0, brow, kb * kBChunks, pol_b);
           if constexpr (MODE == kModeFwd) {
             if constexpr (EPI == MOE_EPI_SWIGLU) {
               // packed: [2 halves][64 rows][64 B]; scales: [4 groups][2 halves][64]
@@ -326,7 +355,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     // ~100 cycles whatever N is, so the reduction of a tile is split among NI
     // issuing warps: issuer j takes the fills f with f % NI == j into its own
     // partial accumulator; the epilogue adds the partials in issuer order.
-    if (lane == 0) {
+    // In a pair only the even CTA issues; its MMAs read the A stages and
+    // token rows of both CTAs and write both accumulators, and its commits
+    // arrive on the barriers of both.
+    if (lane == 0 && rank == 0) {
       const int j = warp - kIssuerWarp0;
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(j * p.acc_cols);
       int st = j, sa = j;                     // stages of the next own fill (f = j, j + NI, ...)
@@ -334,29 +366,40 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       int it = 0;
       int r0 = 0;                             // (first fill of the tile) % NI
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const uint32_t idesc = idesc_bf16_f32(kTileF, decode_tile(p, tile_start, A, t).width,
+      auto commit = [](uint32_t bar) {
+        if constexpr (PAIR) mma_commit_pair(bar, 3); else mma_commit(bar);
+      };
+      auto mma_ts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t accum) {
+        if constexpr (PAIR) mma_bf16_ts_pair(d, a, b, id, accum); else mma_bf16_ts(d, a, b, id, accum);
+      };
+      // Barriers the other CTA of a pair arrives on are waited with cluster scope.
+      auto wait_x = [&](uint32_t bar, uint32_t parity) {
+        if constexpr (PAIR) return mbar_wait_cluster(bar, parity, abort_flag);
+        else return mbar_wait(bar, parity, abort_flag);
+      };
+      for (int t = t_first; t < total && ok; t += t_step, ++it) {
+        const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kTileF : kTileF, tile_at(t).width,
                                               MODE == kModeBwd ? 1u : 0u, 0u);
-        if (!mbar_wait(acc_empty, static_cast<uint32_t>(it & 1) ^ 1u, abort_flag)) { ok = false; break; }
+        if (!wait_x(acc_empty, static_cast<uint32_t>(it & 1) ^ 1u)) { ok = false; break; }
         tc_fence_after();
         uint32_t acc = 0;
         for (int kb = (j - r0 + NI) % NI; kb < nkb; kb += NI) {
           {
-            if (!mbar_wait(full_a(sa), pha, abort_flag)) { ok = false; break; }
+            if (!wait_x(full_a(sa), pha)) { ok = false; break; }
             tc_fence_after();
             const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
             if constexpr (kTmemA) {
               // A stage st: 128 lanes x 64 columns (two BF16 per column): K=16 = 8 columns.
               const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * 64);
               const uint64_t b1 = b0 + (b_chunk >> 4);
-              mma_bf16_ts(d_tmem, a0, b0, idesc, acc);
-              mma_bf16_ts(d_tmem, a0 + 8, b0 + 2, idesc, 1u);
-              mma_bf16_ts(d_tmem, a0 + 16, b0 + 4, idesc, 1u);
-              mma_bf16_ts(d_tmem, a0 + 24, b0 + 6, idesc, 1u);
-              mma_bf16_ts(d_tmem, a0 + 32, b1, idesc, 1u);
-              mma_bf16_ts(d_tmem, a0 + 40, b1 + 2, idesc, 1u);
-              mma_bf16_ts(d_tmem, a0 + 48, b1 + 4, idesc, 1u);
-              mma_bf16_ts(d_tmem, a0 + 56, b1 + 6, idesc, 1u);
+              mma_ts(d_tmem, a0, b0, idesc, acc);
+              mma_ts(d_tmem, a0 + 8, b0 + 2, idesc, 1u);
+              mma_ts(d_tmem, a0 + 16, b0 + 4, idesc, 1u);
+              mma_ts(d_tmem, a0 + 24, b0 + 6, idesc, 1u);
+              mma_ts(d_tmem, a0 + 32, b1, idesc, 1u);
+              mma_ts(d_tmem, a0 + 40, b1 + 2, idesc, 1u);
+              mma_ts(d_tmem, a0 + 48, b1 + 4, idesc, 1u);
+              mma_ts(d_tmem, a0 + 56, b1 + 6, idesc, 1u);
             } else {
               const uint64_t a0 = smem_desc_sw128(A_at(st), 8192, 1024);
               mma_bf16_ss(d_tmem, a0, b0, idesc, acc);
@@ -365,8 +408,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
               mma_bf16_ss(d_tmem, a0 + 384, b0 + 6, idesc, 1u);
             }
             acc = 1u;
-            mma_commit(empty(st));
-            if constexpr (kTmemA) mma_commit(a_free(sa));
+            commit(empty(st));
+            if constexpr (kTmemA) commit(a_free(sa));
           }
           st += NI;
           if (st >= S) st -= S;
@@ -374,10 +417,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           if (sa >= SA) { sa -= SA; pha ^= 1u; }
         }
         r0 = (r0 + nkb) % NI;
-        if (ok) mma_commit(acc_full);         // arrives even when this issuer had no fill
+        if (ok) commit(acc_full);             // arrives even when this issuer had no fill
       }
-      // All MMAs of this CTA done before tensor memory is released.
-      mma_commit(drain_bar);
+      // All MMAs of this CTA (of the pair) done before tensor memory is released.
+      commit(drain_bar);
       mbar_drain(drain_bar, 0);
     }
   } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kLanes * kDqWarpsPerLane) {
@@ -402,7 +445,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     int st = grp, sa = grp;                 // fill ring and A ring positions of the next own fill
     uint32_t ph = 0, pha = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+    for (int t = t_first; t < total && ok; t += t_step) {
       const int kb_first = (grp - r0 + kLanes) % kLanes;
       r0 = (r0 + nkb) % kLanes;
       for (int kb = kb_first; kb < nkb; kb += kLanes) {
@@ -480,7 +523,11 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(full_a(cur_a));
+        if (lane == 0) {
+          // A pair's A stages are waited for by the even CTA's issuers.
+          if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(full_a(cur_a), 0));
+          else mbar_arrive(full_a(cur_a));
+        }
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -495,8 +542,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     static_assert(kMaxIssuers <= 3, "the epilogue sums at most three partial accumulators");
     int it = 0;
     int r0 = 0;                             // (first fill of the tile) % NI
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const Tile tl = decode_tile(p, tile_start, A, t);
+    for (int t = t_first; t < total; t += t_step, ++it) {
+      const Tile tl = tile_at(t);
       // Issuer j wrote its partial in this tile iff one of the tile's nkb
       // fills f has f % NI == j.
       const bool has0 = ((NI - r0) % NI) < nkb;
@@ -535,20 +582,28 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         }
         const int nrows = min(16, tl.row_end - (tl.row0 + c0));
         if constexpr (kGluRows) {
-          // Lanes 0-15 hold gate values, lanes 16-31 the up values of the same
-          // 16 features. Staging row (64 BF16): [0,16) h, [16,32) g, [32,48) u.
+          // Lanes 0-15 hold gate values g, lanes 16-31 the up values u of the
+          // same 16 features (pr = lane & 15). Each lane forms h = silu(g) * u
+          // for 8 of the 16 token columns, gate lanes columns 0-7 and up lanes
+          // 8-15, after swapping the missing operand with lane ^ 16. The code
+          // has no branch, so the eight columns' exponentials, divisions and
+          // shuffles overlap. Staging row (64 BF16): [0,16) h, [16,32) g, [32,48) u.
           const int pr = lane & 15;
           const bool is_gate = lane < 16;
+          const int hrow0 = is_gate ? 0 : 8;
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const float other = __shfl_xor_sync(0xffffffffu, v[jj], 16);
-            uint16_t* row = stg_ptr + jj * 64;
-            if (is_gate) {
-              row[pr] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_f(v[jj]) * other));
-              row[16 + pr] = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
-            } else {
-              row[32 + pr] = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
-            }
+          for (int jj = 0; jj < 8; ++jj) {
+            const float mine = is_gate ? v[jj] : v[jj + 8];
+            const float got = __shfl_xor_sync(0xffffffffu, is_gate ? v[jj + 8] : v[jj], 16);
+            const float g = is_gate ? mine : got;
+            const float u = is_gate ? got : mine;
+            stg_ptr[(hrow0 + jj) * 64 + pr] = __bfloat16_as_ushort(__float2bfloat16_rn(silu_f(g) * u));
+          }
+          if (p.saved) {
+            // g to columns [16, 32) from the gate lanes, u to [32, 48) from the up lanes.
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj)
+              stg_ptr[jj * 64 + 16 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
           }
           __syncwarp();
           // 16 H features of this warp: 32 B per row = 2 chunks; g and u likewise.
@@ -568,20 +623,35 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           __syncwarp();
         } else if constexpr (MODE == kModeBwd && EPI == MOE_EPI_SWIGLU_BWD) {
           const int f = tl.ft * kTileF + fr;      // feature of dh (< K)
+          const bool fok = f < p.F;
+          // saved g of row (row0 + c0 + j) and feature f; its u is K further on
+          const uint16_t* sv = reinterpret_cast<const uint16_t*>(p.saved) +
+                               static_cast<int64_t>(tl.row0 + c0) * (2 * K) + (fok ? f : 0);
           // Staging row: [0,32) dg, [32,64) du of this warp's 32 features.
+          // Four rows at a time: their saved g and u are loaded first (no
+          // branch, so the loads are in flight together), then combined.
 #pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            uint16_t dg = 0, du = 0;
-            if (jj < nrows && f < p.F) {
-              const int64_t rb = static_cast<int64_t>(tl.row0 + c0 + jj) * (2 * K);
-              const float g = __bfloat162float(p.saved[rb + f]);
-              const float u = __bfloat162float(p.saved[rb + K + f]);
-              const float s = sigmoid_f(g);
-              dg = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj] * u * s * (1.0f + g * (1.0f - s))));
-              du = __bfloat16_as_ushort(__float2bfloat16_rn(v[jj] * g * s));
+          for (int h8 = 0; h8 < 16; h8 += 4) {
+            uint16_t gb[4], ub[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const bool ok = fok && (h8 + jj) < nrows;
+              const uint16_t* src = sv + (ok ? (h8 + jj) * (2 * K) : 0);
+              gb[jj] = ok ? __ldg(src) : uint16_t(0);
+              ub[jj] = ok ? __ldg(src + K) : uint16_t(0);
             }
-            stg_ptr[jj * 64 + lane] = dg;
-            stg_ptr[jj * 64 + 32 + lane] = du;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+              const float g = __uint_as_float(static_cast<uint32_t>(gb[jj]) << 16);
+              const float u = __uint_as_float(static_cast<uint32_t>(ub[jj]) << 16);
+              const float s = sigmoid_f(g);
+              const float x = v[h8 + jj];
+              const bool ok = fok && (h8 + jj) < nrows;
+              const uint16_t dg = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(x * u * s * (1.0f + g * (1.0f - s)))) : uint16_t(0);
+              const uint16_t du = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(x * g * s)) : uint16_t(0);
+              stg_ptr[(h8 + jj) * 64 + lane] = dg;
+              stg_ptr[(h8 + jj) * 64 + 32 + lane] = du;
+            }
           }
           __syncwarp();
           const int fb = tl.ft * kTileF + q * 32;
@@ -618,26 +688,37 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(acc_empty, 0));
+        else mbar_arrive(acc_empty);
+      }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  // A pair frees its tensor memory only when the even CTA's MMAs, which write
+  // both CTAs' accumulators, have drained and both epilogues are done.
+  if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
-  if (warp == kIssuerWarp0) tmem_dealloc(tmem_base, p.tmem_cols);
+  if (warp == kIssuerWarp0) {
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, p.tmem_cols);
+    else tmem_dealloc(tmem_base, p.tmem_cols);
+  }
 }
 
 }  // namespace
 
-template <int MODE, int FMT, int EPI, int LANES>
+template <int MODE, int FMT, int EPI, int LANES, int PAIR>
 static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorMap& tw,
                                           const CUtensorMap& ts, const GemmArgs& p, int grid,
                                           size_t smem, cudaStream_t s) {
-  auto k = grouped_qgemm_kernel<MODE, FMT, EPI, LANES>;
-  // Raise the dynamic shared-memory limit once per (device, kernel); later
-  // calls, including ones under stream capture, skip it.
+  auto k = grouped_qgemm_kernel<MODE, FMT, EPI, LANES, PAIR>;
+  // Raise the dynamic shared-memory limit once per (device, kernel) and, for
+  // pairs, count the clusters that can be resident at once; later calls,
+  // including ones under stream capture, skip both.
   static int set_for[64] = {0};
+  static int max_pairs[64] = {0};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -647,35 +728,71 @@ static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorM
     if (err != cudaSuccess) return err;
     set_for[dev] = 227 * 1024;
   }
-  k<<<grid, kThreads, smem, s>>>(tb, tw, ts, p);
-  return cudaGetLastError();
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_pairs[dev] == 0) {
+      cfg.gridDim = dim3(2 * ((grid + 1) / 2));
+      int n = 0;
+      err = cudaOccupancyMaxActiveClusters(&n, k, &cfg);
+      if (err != cudaSuccess) return err;
+      if (n < 1) return cudaErrorInvalidConfiguration;
+      max_pairs[dev] = n;
+    }
+    // Persistent pairs: at most as many as can be resident together.
+    const int pairs = std::max(1, std::min((grid + 1) / 2, max_pairs[dev]));
+    cfg.gridDim = dim3(2 * pairs);
+    err = cudaLaunchKernelEx(&cfg, k, tb, tw, ts, p);
+    if (err != cudaSuccess) return err;
+    return cudaGetLastError();
+  } else {
+    k<<<grid, kThreads, smem, s>>>(tb, tw, ts, p);
+    return cudaGetLastError();
+  }
 }
 
-cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, const CUtensorMap& tb,
-                                 const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
-                                 int grid, size_t smem, cudaStream_t s) {
-#define MOEQ_CASE(M_, F_, E_)                                                          \
-  if (mode == M_ && fmt == F_ && epi == E_)                                            \
-    return lanes == 4 ? launch_grouped_qgemm_t<M_, F_, E_, 4>(tb, tw, ts, p, grid, smem, s) \
-                      : launch_grouped_qgemm_t<M_, F_, E_, 2>(tb, tw, ts, p, grid, smem, s);
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, bool pair,
+                                 const CUtensorMap& tb, const CUtensorMap& tw,
+                                 const CUtensorMap& ts, const GemmArgs& p, int grid, size_t smem,
+                                 cudaStream_t s) {
+#define MOEQ_LANES(M_, F_, E_, P_)                                                          \
+  return lanes == 4 ? launch_grouped_qgemm_t<M_, F_, E_, 4, P_>(tb, tw, ts, p, grid, smem, s) \
+                    : launch_grouped_qgemm_t<M_, F_, E_, 2, P_>(tb, tw, ts, p, grid, smem, s);
+#define MOEQ_CASE(M_, F_, E_)                                                  \
+  if (mode == M_ && fmt == F_ && epi == E_) {                                  \
+    if (pair) { MOEQ_LANES(M_, F_, E_, 1) } else { MOEQ_LANES(M_, F_, E_, 0) } \
+  }
+#define MOEQ_CASE_SINGLE(M_, F_, E_) \
+  if (mode == M_ && fmt == F_ && epi == E_ && !pair) { MOEQ_LANES(M_, F_, E_, 0) }
   if (lanes != 2 && lanes != 4) return cudaErrorInvalidValue;
   MOEQ_CASE(kModeFwd, MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
   MOEQ_CASE(kModeFwd, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU)
   MOEQ_CASE(kModeFwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
   MOEQ_CASE(kModeFwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU)
-  MOEQ_CASE(kModeBwd, MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
-  MOEQ_CASE(kModeBwd, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU_BWD)
-  MOEQ_CASE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
-  MOEQ_CASE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU_BWD)
+  MOEQ_CASE_SINGLE(kModeBwd, MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
+  MOEQ_CASE_SINGLE(kModeBwd, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU_BWD)
+  MOEQ_CASE_SINGLE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
+  MOEQ_CASE_SINGLE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU_BWD)
+#undef MOEQ_CASE_SINGLE
 #undef MOEQ_CASE
+#undef MOEQ_LANES
   return cudaErrorInvalidValue;
 }
 
-uint32_t gemm_stage_bytes(int mode, int BN, int fmt) {
+uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair) {
   const uint32_t el = (fmt == MOE_W_INT4_G32_BF16) ? 2u : 1u;
   uint32_t b;
-  if (mode == kModeFwd)   // B 2 chunks, packed 128 rows x 64 B, scales 4 x 128
-    b = static_cast<uint32_t>(BN) * 256u + 8192u + 512u * el;
+  if (mode == kModeFwd)   // B 2 chunks (BN / 2 rows in a pair), packed 128 rows x 64 B, scales 4 x 128
+    b = static_cast<uint32_t>(pair ? BN / 2 : BN) * 256u + 8192u + 512u * el;
   else                    // B 1 chunk, A 16 KiB, packed 64 rows x 64 B, scales 4 x 64
     b = static_cast<uint32_t>(BN) * 128u + kABytes + 4096u + 256u * el;
   return (b + 1023u) & ~1023u;

@@ -17,8 +17,8 @@ struct GemmArgs {
   const int32_t* num_active;  // [1] number of active experts
   int32_t E, N, K;            // weight stack dims, W[e] is [N][K]
   int32_t M;                  // rows of a / dout / out
-  int32_t BN;                 // token rows per tile (multiple of 16, <= 256)
-  int32_t n_ftiles;           // feature tiles per expert
+  int32_t BN;                 // token rows per tile (multiple of 16, of 32 for pairs; <= 256)
+  int32_t n_ftiles;           // feature tiles per expert (pairs: pair tiles of 2 feature tiles)
   int32_t n_issuers;          // MMA-issuing warps (1..kMaxIssuers), each with a partial accumulator
   int32_t acc_cols;           // TMEM columns per partial accumulator (>= BN, multiple of 32)
   int32_t tmem_cols;          // TMEM columns allocated (power of two, >= 2 * acc_cols)
@@ -33,10 +33,14 @@ struct GemmArgs {
   __nv_bfloat16* saved;       // fwd SwiGLU: written [M][N]; bwd SwiGLU: read [M][2K]
 };
 
-cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, const CUtensorMap& tb,
-                                 const CUtensorMap& tw, const CUtensorMap& ts, const GemmArgs& p,
-                                 int grid, size_t smem, cudaStream_t s);
-uint32_t gemm_stage_bytes(int mode, int BN, int fmt);
+// pair: forward only; a cluster of two CTAs per 256 output features with
+// M = 256 MMAs (BN a multiple of 32, an even number of feature tiles); the
+// grid is clamped to the pairs that can be resident together.
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, bool pair,
+                                 const CUtensorMap& tb, const CUtensorMap& tw,
+                                 const CUtensorMap& ts, const GemmArgs& p, int grid, size_t smem,
+                                 cudaStream_t s);
+uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair);
 uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E);
 // Warp roles, in order: kProdWarps TMA producers, up to kMaxIssuers
 // MMA-issuing warps, kDqWarps dequant warps split into LANES groups (LANES is a
