@@ -6,7 +6,10 @@
 //   forward   x'[p][32b+j] = sum_i x[p][32b+i] * R[e][b][i][j]
 //   backward  dx[p][32b+i] = sum_j dx'[p][32b+j] * R[e][b][i][j]
 //             dR[e][b][i][j] = sum over rows p of expert e of x[p][32b+i] * dx'[p][32b+j]
-// FP32 accumulation; dR is summed in ascending row order by one warp per
+// Both kernels multiply on the warp-level tensor-core MMA (mma.sync m16n8k16:
+// BF16 operands, exact products, FP32 accumulation): the operation moves each
+// element of x once, and 32 multiply-adds per element on the FP32 pipes take
+// longer than that. dR is accumulated in ascending row order by one warp per
 // (expert, block) pair, so it is deterministic.
 #include "launchers.cuh"
 #include "common.cuh"
@@ -15,179 +18,228 @@ namespace moeq {
 
 namespace {
 
-constexpr int kBlocksPerCta = 8;   // 32-column blocks per CTA (one warp each)
+// d (16 x 8, FP32) += a (16 x 16, BF16, row-major) * b (16 x 8, BF16, column-major).
+// Fragments (g = lane / 4, t = lane % 4): a = rows g and g + 8 at k pairs 2t and
+// 2t + 8 ({row g, k 2t}, {row g + 8, k 2t}, {row g, k 2t + 8}, {row g + 8, k 2t + 8});
+// b = column g at k pairs 2t and 2t + 8; d = rows g and g + 8 at columns 2t, 2t + 1.
+// A pair packs the lower k (or column) in the low 16 bits.
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* f) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    f[2 * q] = __uint_as_float(w[q] << 16);
-    f[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+__device__ __forceinline__ uint32_t ldg_u32(const __nv_bfloat16* p) {
+  return __ldg(reinterpret_cast<const unsigned int*>(p));
+}
+
+__device__ __forceinline__ uint32_t ldg_u16(const __nv_bfloat16* p) {
+  return __ldg(reinterpret_cast<const unsigned short*>(p));
+}
+
+// Largest e with offsets[e] <= row, for 0 <= row < offsets[E] (offsets nondecreasing).
+__device__ __forceinline__ int expert_of_row(const int32_t* offsets, int E, int row) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(offsets + mid) <= row) lo = mid; else hi = mid - 1;
   }
+  return lo;
 }
 
-constexpr int kApplyRowGroups = 2;   // 32-row groups per warp of the apply kernel
+constexpr int kApplyGroups = 4;   // 16-row groups per warp task of the apply kernel
 
-// Expert of row `row` (the same row in every lane): the largest e with
-// offsets[e] <= row, which is the number of boundaries offsets[1..E-1] at or
-// below the row (offsets are nondecreasing and offsets[E] = M > row); the
-// lanes count them in parallel.
-__device__ __forceinline__ int warp_expert_of_row(const int32_t* offsets, int E, int row, int lane) {
-  int cnt = 0;
-  for (int e = 1 + lane; e < E; e += 32) cnt += (__ldg(offsets + e) <= row) ? 1 : 0;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  return cnt;
-}
-
-// grid (ceil(M / 64), ceil(K / 256)), 256 threads. Warp w covers column block
-// b = 8 * blockIdx.y + w for 64 rows, 32 at a time (one row per lane): the lane
-// keeps its row's 32 inputs in registers and reads its expert's 32 x 32 block
-// from shared memory (a broadcast when the warp's rows share an expert, the
-// common case since rows are sorted by expert); the block is staged again only
-// when the expert changes. TRANS = 0: x . R, 1: x . R^T.
+// One warp task: 64 rows (four 16-row groups) x one 32-column block b; eight
+// tasks per 256-thread CTA, consecutive tasks on consecutive blocks of the same
+// rows. All four groups' x fragments are loaded first (4 KiB in flight per
+// warp); the expert's R block, as B fragments, stays in registers while the
+// rows' expert does not change. A group whose rows span several experts runs
+// the MMAs once per expert and keeps each row's result from its own expert.
+// TRANS = 0: out = x . R_e; 1: out = x . R_e^T.
 template <int TRANS>
 __global__ void __launch_bounds__(256)
 adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ R,
                      const int32_t* __restrict__ offsets, int E, int M, int K,
                      __nv_bfloat16* __restrict__ out) {
-  __shared__ __align__(16) float rs[kBlocksPerCta][32][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.y * kBlocksPerCta + warp;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int nb = K / 32;
-  if (b >= nb) return;                   // warp-uniform; the warps never sync with each other
-  const int row_base = blockIdx.x * 32 * kApplyRowGroups;
-  if (row_base >= M) return;
-  int e = warp_expert_of_row(offsets, E, row_base, lane);   // expert of the warp's first row
-  int staged = -1;                       // expert whose block is in rs[warp]
-  for (int g = 0; g < kApplyRowGroups; ++g) {
-    const int row = row_base + g * 32 + lane;
-    const bool valid = row < M;
-    if (__ballot_sync(0xffffffffu, valid) == 0) break;
-    // this lane's expert: step forward from the warp's first expert
-    int my_e = -1;
-    if (valid) {
-      my_e = e;
-      while (my_e + 1 < E && __ldg(offsets + my_e + 1) <= row) ++my_e;
+  const int64_t task = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int64_t n_spans = (static_cast<int64_t>(M) + 16 * kApplyGroups - 1) / (16 * kApplyGroups);
+  if (task >= n_spans * nb) return;
+  const int b = static_cast<int>(task % nb);
+  const int span0 = static_cast<int>(task / nb) * 16 * kApplyGroups;
+  uint32_t a[kApplyGroups][2][4];
+#pragma unroll
+  for (int q = 0; q < kApplyGroups; ++q) {
+    const int ra = span0 + 16 * q + g, rb = ra + 8;
+    const bool va = ra < M, vb = rb < M;
+    const __nv_bfloat16* xa = x + static_cast<int64_t>(va ? ra : 0) * K + 32 * b + 2 * t;
+    const __nv_bfloat16* xb = x + static_cast<int64_t>(vb ? rb : 0) * K + 32 * b + 2 * t;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      a[q][s][0] = va ? ldg_u32(xa + 16 * s) : 0u;
+      a[q][s][1] = vb ? ldg_u32(xb + 16 * s) : 0u;
+      a[q][s][2] = va ? ldg_u32(xa + 16 * s + 8) : 0u;
+      a[q][s][3] = vb ? ldg_u32(xb + 16 * s + 8) : 0u;
     }
-    float xv[32];
-    if (valid) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(row) * K + 32 * b);
+  }
+  int cached = -1;
+  uint32_t bf[4][2][2];   // [n tile][k step][b0, b1] of R block (cached, b)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) unpack_bf16x8(__ldg(src + v), xv + 8 * v);
-    } else {
+  for (int q = 0; q < kApplyGroups; ++q) {
+    const int r0 = span0 + 16 * q;
+    if (r0 >= M) break;
+    const int ra = r0 + g, rb = ra + 8;
+    const int e_first = expert_of_row(offsets, E, r0);
+    const int e_last = expert_of_row(offsets, E, min(r0 + 15, M - 1));
+    float res[4][4];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) xv[i] = 0.0f;
-    }
-    float acc[32];
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
-    int pending = my_e;
-    while (true) {
-      const unsigned live = __ballot_sync(0xffffffffu, pending >= 0);
-      if (live == 0) break;
-      const int cur = __shfl_sync(0xffffffffu, pending, __ffs(live) - 1);
-      if (cur != staged) {
-        // stage R[cur][b] (TRANS: its transpose) as rs[warp][i][j] = coefficient
-        // of input i in output j; lane writes column `lane` of row i (no bank conflict)
-        __syncwarp();
-        const __nv_bfloat16* Rb = R + ((static_cast<int64_t>(cur) * nb + b) * 32) * 32;
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i)
-          rs[warp][i][lane] = __bfloat162float(TRANS ? Rb[lane * 32 + i] : Rb[i * 32 + lane]);
-        __syncwarp();
-        staged = cur;
-      }
-      if (pending == cur) {
+      for (int c = 0; c < 4; ++c) res[nt][c] = 0.0f;
+    for (int e = e_first; e <= e_last; ++e) {
+      const int p0 = __ldg(offsets + e), p1 = __ldg(offsets + e + 1);
+      if (p0 == p1) continue;
+      if (e != cached) {
+        const __nv_bfloat16* Rb = R + (static_cast<int64_t>(e) * nb + b) * 1024;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float xi = xv[i];
-          const float4* r4 = reinterpret_cast<const float4*>(&rs[warp][i][0]);
+        for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const float4 c = r4[m];
-            acc[4 * m] = fmaf(xi, c.x, acc[4 * m]);
-            acc[4 * m + 1] = fmaf(xi, c.y, acc[4 * m + 1]);
-            acc[4 * m + 2] = fmaf(xi, c.z, acc[4 * m + 2]);
-            acc[4 * m + 3] = fmaf(xi, c.w, acc[4 * m + 3]);
+          for (int s = 0; s < 2; ++s) {
+            if (TRANS) {
+              // B[k][n] = R[n][k]: row 8 nt + g of R, k pairs 16 s + 2t and + 8
+              const __nv_bfloat16* c = Rb + (8 * nt + g) * 32 + 16 * s + 2 * t;
+              bf[nt][s][0] = ldg_u32(c);
+              bf[nt][s][1] = ldg_u32(c + 8);
+            } else {
+              // B[k][n] = R[k][n]: column 8 nt + g of R, rows 16 s + 2t (+1) and + 8 (+9)
+              const __nv_bfloat16* c = Rb + (16 * s + 2 * t) * 32 + 8 * nt + g;
+              bf[nt][s][0] = ldg_u16(c) | (ldg_u16(c + 32) << 16);
+              bf[nt][s][1] = ldg_u16(c + 256) | (ldg_u16(c + 288) << 16);
+            }
           }
-        }
-        pending = -1;
+        cached = e;
       }
-    }
-    if (valid) {
-      uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(row) * K + 32 * b);
+      const bool ina = ra >= p0 && ra < p1, inb = rb >= p0 && rb < p1;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 o;
-        o.x = pack_bf16x2(acc[8 * v + 0], acc[8 * v + 1]);
-        o.y = pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]);
-        o.z = pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]);
-        o.w = pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]);
-        dst[v] = o;
+      for (int nt = 0; nt < 4; ++nt) {
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        mma16816(d, a[q][0], bf[nt][0][0], bf[nt][0][1]);
+        mma16816(d, a[q][1], bf[nt][1][0], bf[nt][1][1]);
+        if (ina) { res[nt][0] = d[0]; res[nt][1] = d[1]; }
+        if (inb) { res[nt][2] = d[2]; res[nt][3] = d[3]; }
       }
     }
-    // the next group starts from the last expert of this one
-    e = __shfl_sync(0xffffffffu, valid ? my_e : -1, 31);
-    if (e < 0) break;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int col = 32 * b + 8 * nt + 2 * t;
+      if (ra < M)
+        *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(ra) * K + col) = pack_bf16x2(res[nt][0], res[nt][1]);
+      if (rb < M)
+        *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(rb) * K + col) = pack_bf16x2(res[nt][2], res[nt][3]);
+    }
   }
 }
 
-constexpr int kGradRows = 16;   // rows staged per step of the gradient kernel
+constexpr int kGradWarps = 8;     // column blocks per CTA of the gradient kernel (one warp each)
+constexpr int kGradRows = 32;     // rows staged per step
+constexpr int kStageLd = 40;      // staged row length in BF16 (80 bytes: conflict-free ldmatrix)
 
-// grid (E, ceil(K / 256)), 256 threads: dR[e][b] for the 8 column blocks b of this
-// CTA (one warp each) over the rows of expert e, in ascending row order.
-// Lane i owns row i of the 32 x 32 result (32 accumulators).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// grid (E, ceil(K / 256)), 256 threads: dR[e][b] for the 8 column blocks b of
+// this CTA (one warp each) over the rows of expert e, 32 rows per step in
+// ascending order: the warp stages the rows' x and dx' columns of its block in
+// shared memory (rows past the expert as zeros) and forms
+// dR += x^T (32 x 32 rows) . dx' (32 rows x 32): A = x^T and B = dx' both come
+// from the staged row-major tiles through transposing matrix loads.
 __global__ void __launch_bounds__(256)
 adapter_grad_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ dxp,
                     const int32_t* __restrict__ offsets, int K, float* __restrict__ dR) {
-  __shared__ float xs[kBlocksPerCta][kGradRows][33];
-  __shared__ __align__(16) float gs[kBlocksPerCta][kGradRows][32];
+  __shared__ __align__(16) uint16_t xs[kGradWarps][kGradRows][kStageLd];
+  __shared__ __align__(16) uint16_t gs[kGradWarps][kGradRows][kStageLd];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int e = blockIdx.x;
-  const int b = blockIdx.y * kBlocksPerCta + warp;
+  const int b = blockIdx.y * kGradWarps + warp;
   const int nb = K / 32;
   if (b >= nb) return;                   // warp-uniform; the warps never sync with each other
   const int p0 = offsets[e], p1 = offsets[e + 1];
-  float acc[32];
+  float acc[2][4][4];                    // [i tile][j tile][fragment]
 #pragma unroll
-  for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[mi][nt][c] = 0.0f;
+  const uint32_t xs0 = smem_u32(&xs[warp][0][0]);
+  const uint32_t gs0 = smem_u32(&gs[warp][0][0]);
+  // ldmatrix row addresses of this lane: matrix m = lane / 8, its row lane % 8.
+  const int m = lane >> 3, mr = lane & 7;
   for (int c0 = p0; c0 < p1; c0 += kGradRows) {
-    const int n = min(kGradRows, p1 - c0);
-    // lane r < n loads row c0 + r of both operands (64 bytes each)
-    if (lane < n) {
-      const int64_t gi = static_cast<int64_t>(c0 + lane) * K + 32 * b;
-      const uint4* xsrc = reinterpret_cast<const uint4*>(x + gi);
-      const uint4* gsrc = reinterpret_cast<const uint4*>(dxp + gi);
+    // 32 rows x 4 chunks of 16 bytes per operand: four chunks per lane.
+    uint4 vx[4], vg[4];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        float f[8];
-        unpack_bf16x8(__ldg(xsrc + v), f);
+    for (int h = 0; h < 4; ++h) {
+      const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
+      const bool ok = c0 + row < p1;
+      const int64_t gi = static_cast<int64_t>(ok ? c0 + row : p0) * K + 32 * b + 8 * ch;
+      vx[h] = ok ? __ldg(reinterpret_cast<const uint4*>(x + gi)) : make_uint4(0, 0, 0, 0);
+      vg[h] = ok ? __ldg(reinterpret_cast<const uint4*>(dxp + gi)) : make_uint4(0, 0, 0, 0);
+    }
+    __syncwarp();                        // the previous step's matrix loads are done
 #pragma unroll
-        for (int q = 0; q < 8; ++q) xs[warp][lane][8 * v + q] = f[q];
-        unpack_bf16x8(__ldg(gsrc + v), f);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) gs[warp][lane][8 * v + q] = f[q];
-      }
+    for (int h = 0; h < 4; ++h) {
+      const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
+      *reinterpret_cast<uint4*>(&xs[warp][row][8 * ch]) = vx[h];
+      *reinterpret_cast<uint4*>(&gs[warp][row][8 * ch]) = vg[h];
     }
     __syncwarp();
-    for (int r = 0; r < n; ++r) {
-      const float xi = xs[warp][r][lane];
-      const float4* g4 = reinterpret_cast<const float4*>(&gs[warp][r][0]);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const float4 c = g4[m];
-        acc[4 * m] = fmaf(xi, c.x, acc[4 * m]);
-        acc[4 * m + 1] = fmaf(xi, c.y, acc[4 * m + 1]);
-        acc[4 * m + 2] = fmaf(xi, c.z, acc[4 * m + 2]);
-        acc[4 * m + 3] = fmaf(xi, c.w, acc[4 * m + 3]);
+    for (int s = 0; s < kGradRows / 16; ++s) {
+      // A = x^T (i x k): matrices (i 0-7, k 0-7), (i 8-15, k 0-7), (i 0-7, k 8-15),
+      // (i 8-15, k 8-15) of i tile mi, read from the [k][i] tile transposed.
+      uint32_t af[2][4];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        const int krow = 16 * s + 8 * (m >> 1) + mr;
+        const int icol = 16 * mi + 8 * (m & 1);
+        ldsm_x4_trans(xs0 + (krow * kStageLd + icol) * 2, af[mi][0], af[mi][1], af[mi][2], af[mi][3]);
+      }
+      // B = dx' (k x j): matrices (j tile nt, k 0-7), (nt, k 8-15), (nt + 1, k 0-7),
+      // (nt + 1, k 8-15), read from the [k][j] tile transposed.
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        const int krow = 16 * s + 8 * (m & 1) + mr;
+        const int jcol = 8 * (2 * np + (m >> 1));
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4_trans(gs0 + (krow * kStageLd + jcol) * 2, b00, b01, b10, b11);
+#pragma unroll
+        for (int mi = 0; mi < 2; ++mi) {
+          mma16816(acc[mi][2 * np], af[mi], b00, b01);
+          mma16816(acc[mi][2 * np + 1], af[mi], b10, b11);
+        }
       }
     }
-    __syncwarp();
   }
-  float4* dst = reinterpret_cast<float4*>(dR + ((static_cast<int64_t>(e) * nb + b) * 32 + lane) * 32);
+  float* dst = dR + (static_cast<int64_t>(e) * nb + b) * 1024;
 #pragma unroll
-  for (int v = 0; v < 8; ++v) dst[v] = make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+  for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int i = 16 * mi + g, j = 8 * nt + 2 * t;
+      *reinterpret_cast<float2*>(dst + i * 32 + j) = make_float2(acc[mi][nt][0], acc[mi][nt][1]);
+      *reinterpret_cast<float2*>(dst + (i + 8) * 32 + j) = make_float2(acc[mi][nt][2], acc[mi][nt][3]);
+    }
 }
 
 }  // namespace
@@ -196,8 +248,10 @@ cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* of
                                  int M, int K, void* out, bool transpose, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int nb = K / 32;
-  dim3 grid((M + 32 * kApplyRowGroups - 1) / (32 * kApplyRowGroups),
-            (nb + kBlocksPerCta - 1) / kBlocksPerCta);
+  const int64_t spans = (static_cast<int64_t>(M) + 16 * kApplyGroups - 1) / (16 * kApplyGroups);
+  const int64_t ctas = (spans * nb + 7) / 8;
+  if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(ctas));
   if (transpose)
     adapter_apply_kernel<1><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
                                                  static_cast<const __nv_bfloat16*>(R), offsets, E,
@@ -212,7 +266,7 @@ cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* of
 cudaError_t launch_adapter_grad(const void* x, const void* dxp, const int32_t* offsets, int E,
                                 int K, float* dR, cudaStream_t s) {
   const int nb = K / 32;
-  dim3 grid(E, (nb + kBlocksPerCta - 1) / kBlocksPerCta);
+  dim3 grid(E, (nb + kGradWarps - 1) / kGradWarps);
   adapter_grad_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
                                            static_cast<const __nv_bfloat16*>(dxp), offsets, K, dR);
   return cudaGetLastError();
