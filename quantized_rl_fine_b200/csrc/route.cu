@@ -7,9 +7,9 @@
 //
 // Four kernels, no host round trip:
 //  1. route_topk_kernel: one warp per token (2 tokens per warp, 64 per
-//     1024-thread block); k rounds of a warp-wide argmax (ties to the lower
-//     expert id), softmax of the k selected logits, and a per-block expert
-//     histogram in shared memory.
+//     1024-thread block; one token per warp for small launches); k rounds of a
+//     warp-wide argmax (ties to the lower expert id), softmax of the k
+//     selected logits, and a per-block expert histogram in shared memory.
 //  2. route_scan_kernel: one block; per expert, an exclusive scan of the
 //     block histograms (block bases for step 3), then scans over experts for
 //     the offsets, the active list and the chunk table.
@@ -19,6 +19,11 @@
 //     offsets[e] + block_base[e] + rank.
 //  4. permute_rows_kernel: one warp per permuted row copies its token row
 //     with 16-byte loads and stores across the whole grid.
+// Small launches (T <= 1024 and a token-by-expert bit matrix of at most 8192
+// words) replace steps 2 and 3 by route_tail_kernel: one block builds, for
+// every expert, the bit mask of its tokens over all T, and takes counts,
+// offsets and stable ranks from popcounts of those masks; the serial walk
+// over the per-block histograms, and one launch, go away.
 #include "common.cuh"
 #include "launchers.cuh"
 
@@ -29,6 +34,7 @@ namespace {
 constexpr int kRouteTokensPerBlock = 64;
 constexpr int kRouteThreads = 256;
 constexpr int kTopkThreads = 1024;
+constexpr int kTailMaxWords = 8192;   // token-by-expert bit matrix of the single-block tail
 
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
@@ -36,18 +42,22 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 
 // NPER: logits held per lane (>= ceil(E / 32)); the selection loops run over
 // exactly NPER slots.
+// tpb tokens per block (a multiple of 32); block_counts == nullptr skips the
+// per-block histogram.
 template <int NPER>
 __global__ void __launch_bounds__(kTopkThreads)
-route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int tpb,
                   int32_t* __restrict__ topk_idx, float* __restrict__ gates,
                   int32_t* __restrict__ block_counts) {
   extern __shared__ int32_t hist[];   // [E]
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  const bool with_hist = block_counts != nullptr;
+  if (with_hist)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int per_warp = kRouteTokensPerBlock / (kTopkThreads / 32);
+  const int per_warp = tpb / (kTopkThreads / 32);
   for (int u = 0; u < per_warp; ++u) {
-    const int t = blockIdx.x * kRouteTokensPerBlock + warp * per_warp + u;
+    const int t = blockIdx.x * tpb + warp * per_warp + u;
     if (t >= T) break;
     const float* row = logits + static_cast<int64_t>(t) * E;
     float v[NPER];
@@ -79,6 +89,9 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
           bi = oi;
         }
       }
+      // Only rows with NaN logits can leave no candidate; keep the index in
+      // range (their routing is unspecified).
+      bi = min(bi, E - 1);
       if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
       if (lane == j) {
         my_val = bv;
@@ -94,32 +107,25 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
     if (lane < k) {
       topk_idx[static_cast<int64_t>(t) * k + lane] = my_idx;
       gates[static_cast<int64_t>(t) * k + lane] = z / sum;
-      atomicAdd(&hist[my_idx], 1);
+      if (with_hist) atomicAdd(&hist[my_idx], 1);
     }
   }
+  if (!with_hist) return;
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
 }
 
-// One block of 1024 threads, E <= 1024.
-__global__ void __launch_bounds__(1024)
-route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk_size,
-                  int32_t* __restrict__ offsets, int32_t* __restrict__ active,
-                  int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
-                  int32_t* __restrict__ num_chunks) {
+// Block-wide step shared by the scan kernels (blockDim = 1024, E <= 1024):
+// thread e holds the row count of expert e; writes offsets[0..E], the active
+// list (ascending ids), num_active and the chunk table, and returns the
+// exclusive offset of expert e.
+__device__ int scan_experts(int cnt, int E, int chunk_size, int32_t* __restrict__ offsets,
+                            int32_t* __restrict__ active, int32_t* __restrict__ num_active,
+                            int32_t* __restrict__ chunk_offsets, int32_t* __restrict__ num_chunks) {
   __shared__ int32_t ws_cnt[32];
   __shared__ int32_t ws_act[32];
   const int e = threadIdx.x;
-  int cnt = 0;
-  if (e < E) {
-    for (int b = 0; b < nblk; ++b) {
-      const int64_t i = static_cast<int64_t>(b) * E + e;
-      const int c = block_counts[i];
-      block_counts[i] = cnt;      // becomes the block's base inside expert e
-      cnt += c;
-    }
-  }
   const int act = (e < E && cnt > 0) ? 1 : 0;
   const int lane = e & 31, w = e >> 5;
   int xc = cnt, xa = act;
@@ -159,14 +165,88 @@ route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk
     if (act) active[incl_a - 1] = e;
   }
   if (e == E - 1) offsets[E] = incl_c;
-  __syncthreads();
-  const int A = ws_act[(E - 1) >> 5] ;   // inclusive total of the last warp holding an expert
+  const int A = ws_act[(E - 1) >> 5];   // inclusive total of the last warp holding an expert
   const int nch = (A + chunk_size - 1) / chunk_size;
   if (e == 0) {
     *num_active = A;
     *num_chunks = nch;
   }
   for (int c = e; c <= nch; c += blockDim.x) chunk_offsets[c] = min(c * chunk_size, A);
+  return incl_c - cnt;
+}
+
+// One block of 1024 threads, E <= 1024.
+__global__ void __launch_bounds__(1024)
+route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk_size,
+                  int32_t* __restrict__ offsets, int32_t* __restrict__ active,
+                  int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
+                  int32_t* __restrict__ num_chunks) {
+  const int e = threadIdx.x;
+  int cnt = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int64_t i = static_cast<int64_t>(b) * E + e;
+      const int c = block_counts[i];
+      block_counts[i] = cnt;      // becomes the block's base inside expert e
+      cnt += c;
+    }
+  }
+  scan_experts(cnt, E, chunk_size, offsets, active, num_active, chunk_offsets, num_chunks);
+}
+
+// One block of 1024 threads, E <= 1024, W = ceil(T / 32) <= 32 words per
+// expert, E * W <= kTailMaxWords. mask[e][w] bit b is set when token 32 w + b
+// chose expert e; pre[e][w] counts the tokens of expert e in words before w
+// (one warp per expert scans its W word popcounts). The rank of token t in
+// expert e is pre[e][w] + popc(mask[e][w] below bit b), so rows stay in
+// ascending token order inside each expert.
+__global__ void __launch_bounds__(1024)
+route_tail_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int chunk_size,
+                  int32_t* __restrict__ offsets, int32_t* __restrict__ active,
+                  int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
+                  int32_t* __restrict__ num_chunks, int32_t* __restrict__ perm_token,
+                  int32_t* __restrict__ inv_perm) {
+  extern __shared__ uint32_t tail_sm[];
+  __shared__ int32_t cnt_s[1024];
+  __shared__ int32_t off_s[1024];
+  const int W = (T + 31) >> 5;
+  uint32_t* mask = tail_sm;                                   // [E][W]
+  int32_t* pre = reinterpret_cast<int32_t*>(tail_sm + W * E);  // [E][W]
+  for (int i = threadIdx.x; i < W * E; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int n = T * k;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int t = i / k;
+    const int e = __ldg(topk_idx + i);
+    atomicOr(&mask[e * W + (t >> 5)], 1u << (t & 31));
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = warp; e < E; e += 32) {
+    const int c = (lane < W) ? __popc(mask[e * W + lane]) : 0;
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < W) pre[e * W + lane] = x - c;
+    if (lane == 31) cnt_s[e] = x;
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  const int off = scan_experts(e < E ? cnt_s[e] : 0, E, chunk_size, offsets, active, num_active,
+                               chunk_offsets, num_chunks);
+  if (e < E) off_s[e] = off;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int t = i / k;
+    const int ex = __ldg(topk_idx + i);
+    const int w = t >> 5, b = t & 31;
+    const int p = off_s[ex] + pre[ex * W + w] + __popc(mask[ex * W + w] & ((1u << b) - 1u));
+    perm_token[p] = t;
+    inv_perm[i] = p;
+  }
 }
 
 __global__ void __launch_bounds__(kRouteThreads)
@@ -233,12 +313,17 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                          int32_t* active, int32_t* num_active, int32_t* chunk_offsets,
                          int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
                          void* x_perm, int32_t* block_counts, cudaStream_t s) {
-  const int nblk = route_num_blocks(T);
+  const int W = (T + 31) / 32;
+  // Small launches: one token per warp, then the single-block tail.
+  const bool small = W <= 32 && W * E <= kTailMaxWords;
+  const int tpb = small ? kTopkThreads / 32 : kRouteTokensPerBlock;
+  const int nblk = small ? (T + tpb - 1) / tpb : route_num_blocks(T);
+  int32_t* hist_out = small ? nullptr : block_counts;
   const int nper = (E + 31) / 32;
-  const size_t hsm = E * sizeof(int32_t);
-#define MOEQ_TOPK(N_)                                                                         \
-  route_topk_kernel<N_><<<nblk, kTopkThreads, hsm, s>>>(logits, T, E, k, topk_idx, gates,     \
-                                                        block_counts)
+  const size_t hsm = small ? 0 : E * sizeof(int32_t);
+#define MOEQ_TOPK(N_)                                                                           \
+  route_topk_kernel<N_><<<nblk, kTopkThreads, hsm, s>>>(logits, T, E, k, tpb, topk_idx, gates, \
+                                                        hist_out)
   if (nper <= 1) MOEQ_TOPK(1);
   else if (nper <= 2) MOEQ_TOPK(2);
   else if (nper <= 4) MOEQ_TOPK(4);
@@ -249,13 +334,33 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
 #undef MOEQ_TOPK
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, chunk_size, offsets, active,
-                                       num_active, chunk_offsets, num_chunks);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  const size_t sm = 2 * E * sizeof(uint32_t);
-  route_scatter_kernel<<<nblk, kRouteThreads, sm, s>>>(topk_idx, block_counts, offsets, T, E, k,
-                                                       perm_token, inv_perm);
+  if (small) {
+    // The tail's dynamic shared memory may pass 48 KiB: raise the limit once
+    // per device (later calls, including ones under stream capture, skip it).
+    static bool raised[64] = {false};
+    int dev = 0;
+    err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!raised[dev]) {
+      err = cudaFuncSetAttribute(route_tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(2 * kTailMaxWords * sizeof(uint32_t)));
+      if (err != cudaSuccess) return err;
+      raised[dev] = true;
+    }
+    const size_t tsm = 2 * static_cast<size_t>(W) * E * sizeof(uint32_t);
+    route_tail_kernel<<<1, 1024, tsm, s>>>(topk_idx, T, E, k, chunk_size, offsets, active,
+                                           num_active, chunk_offsets, num_chunks, perm_token,
+                                           inv_perm);
+  } else {
+    route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, chunk_size, offsets, active,
+                                         num_active, chunk_offsets, num_chunks);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const size_t sm = 2 * E * sizeof(uint32_t);
+    route_scatter_kernel<<<nblk, kRouteThreads, sm, s>>>(topk_idx, block_counts, offsets, T, E,
+                                                         k, perm_token, inv_perm);
+  }
   err = cudaGetLastError();
   if (err != cudaSuccess || x == nullptr) return err;
   const int M = T * k;
