@@ -25,6 +25,10 @@ TINY_TRAIN = MoEConfig("tiny_train_int4_adapter", E=8, k=2, d=256, f=256, T=96, 
                        swiglu=True, logits="normal", adapter=True, train=True, seed=2001)
 RAGGED_MX = MoEConfig("ragged_mxfp4", E=5, k=3, d=128, f=192, T=37, fmt="mxfp4", swiglu=True,
                       logits="normal", adapter=True, train=True, seed=2002, chunk_size=2)
+# About 150 rows per expert: the backward plans 192-row token tiles (one tile
+# of 160 or more rows per expert), wider than any forward tile.
+WIDE = MoEConfig("wide_int4", E=4, k=2, d=256, f=256, T=300, fmt="int4", swiglu=True,
+                 logits="normal", adapter=True, train=True, seed=2003)
 
 
 def _to(wl, dev):
@@ -195,7 +199,15 @@ def _run_layer_and_compare(cfg, T=None):
         bw = layer.backward(st, wl["dy"], wl["w_gu"], wl["w_d"], adapter=wl.get("adapter"))
         torch.cuda.synchronize()
         rb = O.moe_backward(ref, f64(wl["dy"]), ow["w_gu"], ow["w_d"], R=R)
-        assert np.array_equal(bf16_bits(bw["dy_perm"]), O.bf16_bits_from_values(rb["dy_perm"]))
+        # The gate-scaled scatter rounds g * dy once to BF16: bit-exact given
+        # the same gates. The kernel's gates match the oracle's only within
+        # the routing check's 2e-6, and a one-ulp gate difference moves a few
+        # products across a BF16 rounding boundary, so the expected rows are
+        # the oracle's scatter of the kernel's gates.
+        r = st["routing"]
+        want = O.gather_scaled(f64(wl["dy"]), r.inv_perm.cpu().numpy(), r.gates.cpu().numpy(),
+                               wl["dy"].shape[0], cfg.k)
+        assert np.array_equal(bf16_bits(bw["dy_perm"]), O.bf16_bits_from_values(want))
         assert_close_intermediate(f64(bw["dgu"]), rb["dgu"], "dgu")
         assert_close_final(f64(bw["dx"]), rb["dx"], "dx")
         if cfg.adapter:
@@ -268,5 +280,28 @@ def test_each_lane_count_and_tile_width_matches_the_oracle(monkeypatch, cfg, lan
     inputs and checks each against the oracle."""
     monkeypatch.setenv("MOEQ_LANES", str(lanes))
     monkeypatch.setenv("MOEQ_BN", str(bn))
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("bn", [None, "192"], ids=["planned", "forced192"])
+def test_wide_token_tiles_match_the_oracle(monkeypatch, bn):
+    """Token tiles wider than 96 rows: planned for the backward at about 150
+    rows per expert, and forced for both directions (the forward then runs
+    with one MMA-issuing warp, as two 192-column partials and four A stages
+    do not fit tensor memory)."""
+    if bn is not None:
+        monkeypatch.setenv("MOEQ_BN", bn)
+    _run_layer_and_compare(WIDE)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, WIDE], ids=["int4", "wide_int4"])
+def test_cta_pair_forward_matches_the_oracle(monkeypatch, cfg):
+    """The opt-in CTA-pair forward kernels (clusters of two CTAs, M = 256
+    MMAs issued by the even CTA, each CTA holding half of the token rows)
+    against the oracle; both shapes have an even number of feature tiles in
+    both forward GEMMs, so every forward launch runs on pairs."""
+    monkeypatch.setenv("MOEQ_PAIR", "1")
     _run_layer_and_compare(cfg)
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
