@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(256)
 adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ R,
                      const int32_t* __restrict__ offsets, int E, int M, int K,
                      __nv_bfloat16* __restrict__ out) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int nb = K / 32;
@@ -165,6 +167,8 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
 __global__ void __launch_bounds__(256)
 adapter_grad_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ dxp,
                     const int32_t* __restrict__ offsets, int K, float* __restrict__ dR) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   __shared__ __align__(16) uint16_t xs[kGradWarps][kGradRows][kStageLd];
   __shared__ __align__(16) uint16_t gs[kGradWarps][kGradRows][kStageLd];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -252,24 +256,19 @@ cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* of
   const int64_t ctas = (spans * nb + 7) / 8;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(ctas));
-  if (transpose)
-    adapter_apply_kernel<1><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                 static_cast<const __nv_bfloat16*>(R), offsets, E,
-                                                 M, K, static_cast<__nv_bfloat16*>(out));
-  else
-    adapter_apply_kernel<0><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                 static_cast<const __nv_bfloat16*>(R), offsets, E,
-                                                 M, K, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_pdl(transpose ? adapter_apply_kernel<1> : adapter_apply_kernel<0>, grid, dim3(256),
+                    0, s, static_cast<const __nv_bfloat16*>(x),
+                    static_cast<const __nv_bfloat16*>(R), offsets, E, M, K,
+                    static_cast<__nv_bfloat16*>(out));
 }
 
 cudaError_t launch_adapter_grad(const void* x, const void* dxp, const int32_t* offsets, int E,
                                 int K, float* dR, cudaStream_t s) {
   const int nb = K / 32;
   dim3 grid(E, (nb + kGradWarps - 1) / kGradWarps);
-  adapter_grad_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                           static_cast<const __nv_bfloat16*>(dxp), offsets, K, dR);
-  return cudaGetLastError();
+  return launch_pdl(adapter_grad_kernel, grid, dim3(256), 0, s,
+                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dxp),
+                    offsets, K, dR);
 }
 
 }  // namespace moeq

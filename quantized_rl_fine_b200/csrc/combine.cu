@@ -39,6 +39,8 @@ __device__ __forceinline__ uint32_t bf16_of_product(float g, float x) {
 __global__ void combine_kernel(const uint4* __restrict__ rows, const int32_t* __restrict__ inv_perm,
                                const float* __restrict__ gates, int T, int k, int64_t dvec,
                                uint4* __restrict__ out) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -68,6 +70,8 @@ __global__ void combine_kernel(const uint4* __restrict__ rows, const int32_t* __
 __global__ void scatter_kernel(const uint4* __restrict__ rows, const int32_t* __restrict__ inv_perm,
                                const float* __restrict__ gates, int T, int k, int64_t dvec,
                                uint4* __restrict__ out) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -96,14 +100,9 @@ cudaError_t launch_combine(const void* rows, const int32_t* inv_perm, const floa
                            int k, int64_t D, void* out, int mode, cudaStream_t s) {
   const int warps = 8;
   const int blocks = (T + warps - 1) / warps;
-  if (mode == 0) {
-    combine_kernel<<<blocks, warps * 32, 0, s>>>(static_cast<const uint4*>(rows), inv_perm, gates,
-                                                 T, k, D / 8, static_cast<uint4*>(out));
-  } else {
-    scatter_kernel<<<blocks, warps * 32, 0, s>>>(static_cast<const uint4*>(rows), inv_perm, gates,
-                                                 T, k, D / 8, static_cast<uint4*>(out));
-  }
-  return cudaGetLastError();
+  return launch_pdl(mode == 0 ? combine_kernel : scatter_kernel, dim3(blocks), dim3(warps * 32), 0,
+                    s, static_cast<const uint4*>(rows), inv_perm, gates, T, k, D / 8,
+                    static_cast<uint4*>(out));
 }
 
 }  // namespace moeq

@@ -13,6 +13,40 @@
 namespace moeq {
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel of the library is launched with
+// it allowed, so its launch and prologue overlap the end of the previous
+// kernel on the stream; each kernel calls grid_dependency_wait() before its
+// first access to global memory that earlier work on the stream may write or
+// read (the wait returns once every earlier grid has completed and its writes
+// are visible, and at once when there is no such dependency), and then
+// grid_dependents_launch() to let the next kernel start its own prologue.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// ---------------------------------------------------------------------------
 // Device error word and wait budget
 // ---------------------------------------------------------------------------
 

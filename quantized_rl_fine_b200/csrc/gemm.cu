@@ -277,6 +277,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touches only this CTA's shared and tensor memory; the
+  // routing tables and operands below come from earlier kernels.
+  grid_dependency_wait();
+  grid_dependents_launch();
 
   const int A = build_tile_list(p, tile_start, warp_tot);
   const int total = tile_start[A];
@@ -730,11 +734,13 @@ static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorM
   }
   if constexpr (PAIR) {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -751,12 +757,12 @@ static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorM
     // Persistent pairs: at most as many as can be resident together.
     const int pairs = std::max(1, std::min((grid + 1) / 2, max_pairs[dev]));
     cfg.gridDim = dim3(2 * pairs);
+    cfg.numAttrs = 2;
     err = cudaLaunchKernelEx(&cfg, k, tb, tw, ts, p);
     if (err != cudaSuccess) return err;
     return cudaGetLastError();
   } else {
-    k<<<grid, kThreads, smem, s>>>(tb, tw, ts, p);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(grid), dim3(kThreads), smem, s, tb, tw, ts, p);
   }
 }
 

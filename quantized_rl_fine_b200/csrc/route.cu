@@ -50,6 +50,8 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int tpb
                   int32_t* __restrict__ topk_idx, float* __restrict__ gates,
                   int32_t* __restrict__ block_counts) {
   extern __shared__ int32_t hist[];   // [E]
+  grid_dependency_wait();
+  grid_dependents_launch();
   const bool with_hist = block_counts != nullptr;
   if (with_hist)
     for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
@@ -181,6 +183,8 @@ route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk
                   int32_t* __restrict__ offsets, int32_t* __restrict__ active,
                   int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
                   int32_t* __restrict__ num_chunks) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int e = threadIdx.x;
   int cnt = 0;
   if (e < E) {
@@ -197,7 +201,9 @@ route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk
 // One block of 1024 threads, E <= 1024, W = ceil(T / 32) <= 32 words per
 // expert, E * W <= kTailMaxWords. mask[e][w] bit b is set when token 32 w + b
 // chose expert e; pre[e][w] counts the tokens of expert e in words before w
-// (one warp per expert scans its W word popcounts). The rank of token t in
+// (one warp per expert scans its W word popcounts). Rows of the two tables
+// are W + 1 words apart, so that the entries of one word index for different
+// experts fall in different shared-memory banks. The rank of token t in
 // expert e is pre[e][w] + popc(mask[e][w] below bit b), so rows stay in
 // ascending token order inside each expert.
 __global__ void __launch_bounds__(1024)
@@ -206,31 +212,34 @@ route_tail_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int
                   int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
                   int32_t* __restrict__ num_chunks, int32_t* __restrict__ perm_token,
                   int32_t* __restrict__ inv_perm) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   extern __shared__ uint32_t tail_sm[];
   __shared__ int32_t cnt_s[1024];
   __shared__ int32_t off_s[1024];
   const int W = (T + 31) >> 5;
-  uint32_t* mask = tail_sm;                                   // [E][W]
-  int32_t* pre = reinterpret_cast<int32_t*>(tail_sm + W * E);  // [E][W]
-  for (int i = threadIdx.x; i < W * E; i += blockDim.x) mask[i] = 0u;
+  const int WP = W + 1;                                        // row pitch in words
+  uint32_t* mask = tail_sm;                                    // [E][WP]
+  int32_t* pre = reinterpret_cast<int32_t*>(tail_sm + WP * E);  // [E][WP]
+  for (int i = threadIdx.x; i < WP * E; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
   const int n = T * k;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int t = i / k;
     const int e = __ldg(topk_idx + i);
-    atomicOr(&mask[e * W + (t >> 5)], 1u << (t & 31));
+    atomicOr(&mask[e * WP + (t >> 5)], 1u << (t & 31));
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = warp; e < E; e += 32) {
-    const int c = (lane < W) ? __popc(mask[e * W + lane]) : 0;
+    const int c = (lane < W) ? __popc(mask[e * WP + lane]) : 0;
     int x = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += y;
     }
-    if (lane < W) pre[e * W + lane] = x - c;
+    if (lane < W) pre[e * WP + lane] = x - c;
     if (lane == 31) cnt_s[e] = x;
   }
   __syncthreads();
@@ -243,7 +252,7 @@ route_tail_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int
     const int t = i / k;
     const int ex = __ldg(topk_idx + i);
     const int w = t >> 5, b = t & 31;
-    const int p = off_s[ex] + pre[ex * W + w] + __popc(mask[ex * W + w] & ((1u << b) - 1u));
+    const int p = off_s[ex] + pre[ex * WP + w] + __popc(mask[ex * WP + w] & ((1u << b) - 1u));
     perm_token[p] = t;
     inv_perm[i] = p;
   }
@@ -253,6 +262,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ block_base,
                      const int32_t* __restrict__ offsets, int T, int E, int k,
                      int32_t* __restrict__ perm_token, int32_t* __restrict__ inv_perm) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   extern __shared__ uint32_t sm[];      // lo[E], hi[E]
   uint32_t* lo = sm;
   uint32_t* hi = sm + E;
@@ -286,6 +297,8 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
 __global__ void __launch_bounds__(256)
 permute_rows_kernel(const int32_t* __restrict__ perm_token, int M, const uint4* __restrict__ x,
                     uint4* __restrict__ x_perm, int64_t row_vec) {
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (p >= M) return;
@@ -321,18 +334,18 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
   int32_t* hist_out = small ? nullptr : block_counts;
   const int nper = (E + 31) / 32;
   const size_t hsm = small ? 0 : E * sizeof(int32_t);
-#define MOEQ_TOPK(N_)                                                                           \
-  route_topk_kernel<N_><<<nblk, kTopkThreads, hsm, s>>>(logits, T, E, k, tpb, topk_idx, gates, \
-                                                        hist_out)
-  if (nper <= 1) MOEQ_TOPK(1);
-  else if (nper <= 2) MOEQ_TOPK(2);
-  else if (nper <= 4) MOEQ_TOPK(4);
-  else if (nper <= 8) MOEQ_TOPK(8);
-  else if (nper <= 12) MOEQ_TOPK(12);
-  else if (nper <= 16) MOEQ_TOPK(16);
-  else MOEQ_TOPK(32);
+#define MOEQ_TOPK(N_)                                                                  \
+  launch_pdl(route_topk_kernel<N_>, dim3(nblk), dim3(kTopkThreads), hsm, s, logits, T, E, k, \
+             tpb, topk_idx, gates, hist_out)
+  cudaError_t err;
+  if (nper <= 1) err = MOEQ_TOPK(1);
+  else if (nper <= 2) err = MOEQ_TOPK(2);
+  else if (nper <= 4) err = MOEQ_TOPK(4);
+  else if (nper <= 8) err = MOEQ_TOPK(8);
+  else if (nper <= 12) err = MOEQ_TOPK(12);
+  else if (nper <= 16) err = MOEQ_TOPK(16);
+  else err = MOEQ_TOPK(32);
 #undef MOEQ_TOPK
-  cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (small) {
     // The tail's dynamic shared memory may pass 48 KiB: raise the limit once
@@ -344,29 +357,28 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!raised[dev]) {
       err = cudaFuncSetAttribute(route_tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(2 * kTailMaxWords * sizeof(uint32_t)));
+                                 static_cast<int>(2 * (kTailMaxWords + 1024) * sizeof(uint32_t)));
       if (err != cudaSuccess) return err;
       raised[dev] = true;
     }
-    const size_t tsm = 2 * static_cast<size_t>(W) * E * sizeof(uint32_t);
-    route_tail_kernel<<<1, 1024, tsm, s>>>(topk_idx, T, E, k, chunk_size, offsets, active,
-                                           num_active, chunk_offsets, num_chunks, perm_token,
-                                           inv_perm);
+    const size_t tsm = 2 * static_cast<size_t>(W + 1) * E * sizeof(uint32_t);
+    err = launch_pdl(route_tail_kernel, dim3(1), dim3(1024), tsm, s, topk_idx, T, E, k,
+                     chunk_size, offsets, active, num_active, chunk_offsets, num_chunks,
+                     perm_token, inv_perm);
   } else {
-    route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nblk, E, chunk_size, offsets, active,
-                                         num_active, chunk_offsets, num_chunks);
-    err = cudaGetLastError();
+    err = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, s, block_counts, nblk, E,
+                     chunk_size, offsets, active, num_active, chunk_offsets, num_chunks);
     if (err != cudaSuccess) return err;
     const size_t sm = 2 * E * sizeof(uint32_t);
-    route_scatter_kernel<<<nblk, kRouteThreads, sm, s>>>(topk_idx, block_counts, offsets, T, E,
-                                                         k, perm_token, inv_perm);
+    err = launch_pdl(route_scatter_kernel, dim3(nblk), dim3(kRouteThreads), sm, s,
+                     static_cast<const int32_t*>(topk_idx), static_cast<const int32_t*>(block_counts),
+                     static_cast<const int32_t*>(offsets), T, E, k, perm_token, inv_perm);
   }
-  err = cudaGetLastError();
   if (err != cudaSuccess || x == nullptr) return err;
   const int M = T * k;
-  permute_rows_kernel<<<(M + 7) / 8, 256, 0, s>>>(perm_token, M, static_cast<const uint4*>(x),
-                                                  static_cast<uint4*>(x_perm), d / 8);
-  return cudaGetLastError();
+  return launch_pdl(permute_rows_kernel, dim3((M + 7) / 8), dim3(256), 0, s,
+                    static_cast<const int32_t*>(perm_token), M, static_cast<const uint4*>(x),
+                    static_cast<uint4*>(x_perm), d / 8);
 }
 
 }  // namespace moeq
