@@ -24,6 +24,8 @@
 // every expert, the bit mask of its tokens over all T, and takes counts,
 // offsets and stable ranks from popcounts of those masks; the serial walk
 // over the per-block histograms, and one launch, go away.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launchers.cuh"
 
@@ -34,7 +36,8 @@ namespace {
 constexpr int kRouteTokensPerBlock = 64;
 constexpr int kRouteThreads = 256;
 constexpr int kTopkThreads = 1024;
-constexpr int kTailMaxWords = 8192;   // token-by-expert bit matrix of the single-block tail
+constexpr int kTailMaxWords = 8192;   // token-by-expert bit matrix of the routing tail
+constexpr int kTailRowsPerBlock = 256; // permuted rows a tail block writes and copies
 
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
@@ -124,7 +127,8 @@ route_topk_kernel(const float* __restrict__ logits, int T, int E, int k, int tpb
 // exclusive offset of expert e.
 __device__ int scan_experts(int cnt, int E, int chunk_size, int32_t* __restrict__ offsets,
                             int32_t* __restrict__ active, int32_t* __restrict__ num_active,
-                            int32_t* __restrict__ chunk_offsets, int32_t* __restrict__ num_chunks) {
+                            int32_t* __restrict__ chunk_offsets, int32_t* __restrict__ num_chunks,
+                            bool write = true) {
   __shared__ int32_t ws_cnt[32];
   __shared__ int32_t ws_act[32];
   const int e = threadIdx.x;
@@ -162,6 +166,7 @@ __device__ int scan_experts(int cnt, int E, int chunk_size, int32_t* __restrict_
   __syncthreads();
   const int incl_c = xc + (w > 0 ? ws_cnt[w - 1] : 0);
   const int incl_a = xa + (w > 0 ? ws_act[w - 1] : 0);
+  if (!write) return incl_c - cnt;
   if (e < E) {
     offsets[e] = incl_c - cnt;
     if (act) active[incl_a - 1] = e;
@@ -198,7 +203,7 @@ route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk
   scan_experts(cnt, E, chunk_size, offsets, active, num_active, chunk_offsets, num_chunks);
 }
 
-// One block of 1024 threads, E <= 1024, W = ceil(T / 32) <= 32 words per
+// Blocks of 1024 threads, E <= 1024, W = ceil(T / 32) <= 32 words per
 // expert, E * W <= kTailMaxWords. mask[e][w] bit b is set when token 32 w + b
 // chose expert e; pre[e][w] counts the tokens of expert e in words before w
 // (one warp per expert scans its W word popcounts). Rows of the two tables
@@ -206,24 +211,33 @@ route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E, int chunk
 // experts fall in different shared-memory banks. The rank of token t in
 // expert e is pre[e][w] + popc(mask[e][w] below bit b), so rows stay in
 // ascending token order inside each expert.
+// Every block builds the tables (a few microseconds of shared-memory work);
+// block 0 writes the offsets, the active list and the chunk table, and block
+// b writes the permutation entries of the permuted rows [p0, p1) it owns and,
+// when x is given, copies those rows (x_perm[p] = x[perm_token[p]]), so the
+// row copy needs no launch of its own.
 __global__ void __launch_bounds__(1024)
 route_tail_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int chunk_size,
                   int32_t* __restrict__ offsets, int32_t* __restrict__ active,
                   int32_t* __restrict__ num_active, int32_t* __restrict__ chunk_offsets,
                   int32_t* __restrict__ num_chunks, int32_t* __restrict__ perm_token,
-                  int32_t* __restrict__ inv_perm) {
+                  int32_t* __restrict__ inv_perm, const uint4* __restrict__ x,
+                  uint4* __restrict__ x_perm, int64_t row_vec) {
   grid_dependency_wait();
   grid_dependents_launch();
   extern __shared__ uint32_t tail_sm[];
   __shared__ int32_t cnt_s[1024];
   __shared__ int32_t off_s[1024];
+  __shared__ int32_t tok_s[kTailRowsPerBlock];
   const int W = (T + 31) >> 5;
   const int WP = W + 1;                                        // row pitch in words
   uint32_t* mask = tail_sm;                                    // [E][WP]
   int32_t* pre = reinterpret_cast<int32_t*>(tail_sm + WP * E);  // [E][WP]
+  const int n = T * k;
+  const int per = (n + gridDim.x - 1) / gridDim.x;             // permuted rows per block
+  const int p0 = min(n, static_cast<int>(blockIdx.x) * per), p1 = min(n, p0 + per);
   for (int i = threadIdx.x; i < WP * E; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
-  const int n = T * k;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const int t = i / k;
     const int e = __ldg(topk_idx + i);
@@ -233,19 +247,19 @@ route_tail_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = warp; e < E; e += 32) {
     const int c = (lane < W) ? __popc(mask[e * WP + lane]) : 0;
-    int x = c;
+    int xs = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
+      const int y = __shfl_up_sync(0xffffffffu, xs, o);
+      if (lane >= o) xs += y;
     }
-    if (lane < W) pre[e * WP + lane] = x - c;
-    if (lane == 31) cnt_s[e] = x;
+    if (lane < W) pre[e * WP + lane] = xs - c;
+    if (lane == 31) cnt_s[e] = xs;
   }
   __syncthreads();
   const int e = threadIdx.x;
   const int off = scan_experts(e < E ? cnt_s[e] : 0, E, chunk_size, offsets, active, num_active,
-                               chunk_offsets, num_chunks);
+                               chunk_offsets, num_chunks, blockIdx.x == 0);
   if (e < E) off_s[e] = off;
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -253,8 +267,27 @@ route_tail_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int
     const int ex = __ldg(topk_idx + i);
     const int w = t >> 5, b = t & 31;
     const int p = off_s[ex] + pre[ex * WP + w] + __popc(mask[ex * WP + w] & ((1u << b) - 1u));
-    perm_token[p] = t;
-    inv_perm[i] = p;
+    if (p >= p0 && p < p1) {
+      perm_token[p] = t;
+      inv_perm[i] = p;
+      tok_s[p - p0] = t;
+    }
+  }
+  if (x == nullptr) return;
+  __syncthreads();
+  // One warp per owned row, 16-byte moves, four loads in flight per lane.
+  for (int r = warp; r < p1 - p0; r += 32) {
+    const uint4* src = x + static_cast<int64_t>(tok_s[r]) * row_vec;
+    uint4* dst = x_perm + static_cast<int64_t>(p0 + r) * row_vec;
+    int64_t c = lane;
+    for (; c + 96 < row_vec; c += 128) {
+      const uint4 a0 = src[c], a1 = src[c + 32], a2 = src[c + 64], a3 = src[c + 96];
+      dst[c] = a0;
+      dst[c + 32] = a1;
+      dst[c + 64] = a2;
+      dst[c + 96] = a3;
+    }
+    for (; c < row_vec; c += 32) dst[c] = src[c];
   }
 }
 
@@ -362,9 +395,22 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
       raised[dev] = true;
     }
     const size_t tsm = 2 * static_cast<size_t>(W + 1) * E * sizeof(uint32_t);
-    err = launch_pdl(route_tail_kernel, dim3(1), dim3(1024), tsm, s, topk_idx, T, E, k,
-                     chunk_size, offsets, active, num_active, chunk_offsets, num_chunks,
-                     perm_token, inv_perm);
+    // With x, one block per SM (at least enough for kTailRowsPerBlock rows
+    // each) shares the row copy; without it one block does the tail alone.
+    const int M = T * k;
+    int blocks = 1;
+    if (x != nullptr) {
+      int dev_sms = 148;
+      cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev);
+      blocks = std::max(1, std::min(dev_sms, (M + 7) / 8));
+      blocks = std::max(blocks, (M + kTailRowsPerBlock - 1) / kTailRowsPerBlock);
+    } else if (M > kTailRowsPerBlock) {
+      blocks = (M + kTailRowsPerBlock - 1) / kTailRowsPerBlock;
+    }
+    return launch_pdl(route_tail_kernel, dim3(blocks), dim3(1024), tsm, s,
+                      static_cast<const int32_t*>(topk_idx), T, E, k, chunk_size, offsets,
+                      active, num_active, chunk_offsets, num_chunks, perm_token, inv_perm,
+                      static_cast<const uint4*>(x), static_cast<uint4*>(x_perm), d / 8);
   } else {
     err = launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, s, block_counts, nblk, E,
                      chunk_size, offsets, active, num_active, chunk_offsets, num_chunks);
