@@ -364,7 +364,11 @@ def _step_fn(cfg, chunk):
 
 
 def _launches_per_step(cfg):
-    route = 4
+    # routing: top-k and the tail (which also copies the rows) for launches of
+    # at most 1024 tokens whose token-by-expert bit matrix fits 8192 words;
+    # else top-k, scan, scatter and the row copy
+    words = (cfg.T + 31) // 32
+    route = 2 if words <= 32 and words * cfg.E <= 8192 else 4
     if not cfg.swiglu:
         return route + 1
     n = route + 2 + 1                           # gate/up, down, combine
