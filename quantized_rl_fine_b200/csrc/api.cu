@@ -211,7 +211,12 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
       }
     }
     pl.tmem_cols = 512;
+    // MOEQ_STAGES caps the shared-memory ring (tuning only).
     int stages = 16;
+    if (const char* env = getenv("MOEQ_STAGES")) {
+      const int v = atoi(env);
+      if (v >= L && v <= 16 && v % L == 0) stages = v;
+    }
     while (stages > L && !fits(stages, pl.a_stages)) stages -= L;
     pl.stages = stages;
   } else {

@@ -254,7 +254,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       mbar_init(empty(s), 1);
     }
     for (int s = 0; s < SA; ++s) {
-      mbar_init(full_a(s), PAIR ? 2 * kDqWarpsPerLane : kDqWarpsPerLane);
+      // A pair's odd CTA relays its dequant arrivals to the even CTA with one
+      // remote arrival per stage (its own warps arrive locally).
+      mbar_init(full_a(s), (PAIR && rank == 0) ? kDqWarpsPerLane + 1 : kDqWarpsPerLane);
       mbar_init(a_free(s), 1);
     }
     mbar_init(acc_full, p.n_issuers);
@@ -354,6 +356,25 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       }
     }
   } else if (warp >= kIssuerWarp0 && warp < kIssuerWarp0 + NI) {
+    if constexpr (PAIR) {
+      // -------------------------------------------------------- pair relay
+      // The odd CTA issues no MMA. One thread of its first issuer warp waits
+      // for each A stage of this CTA to be complete (its dequant warps
+      // arrive locally) and passes that on with a single arrival on the even
+      // CTA's barrier of the stage.
+      if (rank == 1 && warp == kIssuerWarp0 && lane == 0) {
+        int sa = 0;
+        uint32_t pha = 0;
+        bool ok = true;
+        for (int t = t_first; t < total && ok; t += t_step) {
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!mbar_wait(full_a(sa), pha, abort_flag)) { ok = false; break; }
+            mbar_arrive_cluster(cluster_addr(full_a(sa), 0));
+            if (++sa == SA) { sa = 0; pha ^= 1u; }
+          }
+        }
+      }
+    }
     // ------------------------------------------------------------ MMA issuers
     // One thread issuing tcgen05.mma sustains only about one instruction per
     // ~100 cycles whatever N is, so the reduction of a tile is split among NI
@@ -529,8 +550,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         __syncwarp();
         if (lane == 0) {
           // A pair's A stages are waited for by the even CTA's issuers.
-          if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(full_a(cur_a), 0));
-          else mbar_arrive(full_a(cur_a));
+          mbar_arrive(full_a(cur_a));
         }
       }
     }
@@ -632,20 +652,20 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           const uint16_t* sv = reinterpret_cast<const uint16_t*>(p.saved) +
                                static_cast<int64_t>(tl.row0 + c0) * (2 * K) + (fok ? f : 0);
           // Staging row: [0,32) dg, [32,64) du of this warp's 32 features.
-          // Four rows at a time: their saved g and u are loaded first (no
+          // Two rows at a time: their saved g and u are loaded first (no
           // branch, so the loads are in flight together), then combined.
 #pragma unroll
-          for (int h8 = 0; h8 < 16; h8 += 4) {
-            uint16_t gb[4], ub[4];
+          for (int h8 = 0; h8 < 16; h8 += 2) {
+            uint16_t gb[2], ub[2];
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
               const bool ok = fok && (h8 + jj) < nrows;
               const uint16_t* src = sv + (ok ? (h8 + jj) * (2 * K) : 0);
               gb[jj] = ok ? __ldg(src) : uint16_t(0);
               ub[jj] = ok ? __ldg(src + K) : uint16_t(0);
             }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < 2; ++jj) {
               const float g = __uint_as_float(static_cast<uint32_t>(gb[jj]) << 16);
               const float u = __uint_as_float(static_cast<uint32_t>(ub[jj]) << 16);
               const float s = sigmoid_f(g);
