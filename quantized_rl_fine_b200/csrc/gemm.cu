@@ -3,8 +3,9 @@
 // Orbit article, "Active-expert-chunked dequantization": the experts chosen
 // by the router are taken in fixed-size chunks, their 4-bit weights are
 // dequantized and a grouped GEMM runs over them. Here the dequantization
-// happens inside the GEMM kernel, tile by tile, into shared memory; no BF16
-// weight is ever written to global memory. The DeepSeek-V4 paragraph of the
+// happens inside the GEMM kernel, tile by tile, into tensor memory (forward)
+// or shared memory (backward); no BF16 weight is ever written to global
+// memory. The DeepSeek-V4 paragraph of the
 // same section gives the backward form: only the activation gradient is
 // formed, the frozen base gets none.
 //
@@ -20,14 +21,19 @@
 //
 // The reduction is walked in fills of 128 (forward) or 64 (backward)
 // elements. Fill f of the CTA belongs to pipeline lane f % kLanes, whose
-// dequant group (four warps, one per tensor-memory lane quarter) turns its
-// packed codes into BF16 in registers and then into the A stage; producer
-// warp f % kProdWarps issues its copies (token rows, packed weights, group
-// scales) into a shared-memory stage, and MMA-issuing warp f % n_issuers
-// accumulates it into that issuer's partial accumulator. One issuing thread
-// sustains only about one tcgen05.mma per 70-150 cycles, so splitting the
-// reduction across issuers is what keeps the tensor core fed at small N. An epilogue warpgroup sums the partials in issuer order and writes
+// dequant group (four or eight warps covering the four tensor-memory lane
+// quarters) turns its packed codes into BF16 in registers and then into the A
+// stage; producer warp f % kProdWarps issues its copies (token rows, packed
+// weights, group scales) into a shared-memory stage, and MMA-issuing warp
+// f % n_issuers accumulates it into that issuer's partial accumulator. One
+// issuing thread sustains only about one tcgen05.mma per 70-200 cycles, so
+// splitting the reduction across issuers is what keeps the tensor core fed at
+// small N. An epilogue warpgroup sums the partials in issuer order and writes
 // BF16 (plain, SwiGLU with the saved gate/up, or the SwiGLU backward).
+//
+// The PAIR instantiations (forward, opt-in) run clusters of two CTAs on 256
+// output features with M = 256 MMAs issued by the even CTA; each CTA holds
+// its own weight rows and half of the token rows.
 // Every wait is bounded; on a timeout the kernel records a device error,
 // lets its in-flight copies and MMAs finish (again bounded), frees tensor
 // memory and returns.
@@ -548,10 +554,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           fence_proxy_async_smem();
         }
         __syncwarp();
-        if (lane == 0) {
-          // A pair's A stages are waited for by the even CTA's issuers.
-          mbar_arrive(full_a(cur_a));
-        }
+        // (In a pair the odd CTA's relay thread passes this stage on.)
+        if (lane == 0) mbar_arrive(full_a(cur_a));
       }
     }
   } else if (warp >= kEpiWarp0) {
