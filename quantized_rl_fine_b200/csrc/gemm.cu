@@ -236,10 +236,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   auto empty = [&](int s) { return bars + 8u * (S + s); };
   auto full_a = [&](int s) { return bars + 8u * (2 * S + s); };
   auto a_free = [&](int s) { return bars + 8u * (2 * S + SA + s); };
-  const uint32_t acc_full = bars + 8u * (2 * S + 2 * SA);
-  const uint32_t acc_empty = bars + 8u * (2 * S + 2 * SA + 1);
-  const uint32_t drain_bar = bars + 8u * (2 * S + 2 * SA + 2);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (2 * S + 2 * SA + 3));
+  // Accumulator handoff: one pair of barriers per pipeline (two with tile
+  // pipelines, else only the first is used).
+  auto acc_full = [&](int q) { return bars + 8u * (2 * S + 2 * SA + q); };
+  auto acc_empty = [&](int q) { return bars + 8u * (2 * S + 2 * SA + 2 + q); };
+  const uint32_t drain_bar = bars + 8u * (2 * S + 2 * SA + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (2 * S + 2 * SA + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* warp_tot = reinterpret_cast<int32_t*>(tmem_slot + 4);          // [32]
   int32_t* tile_start = warp_tot + 32;                                      // [E + 1]
@@ -253,6 +255,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  // Tile pipelines (forward; two lanes, two issuers, two producers): the
+  // CTA's i-th tile belongs to pipeline i % 2 as a whole (its producer,
+  // dequant lane and issuer, which accumulates all of its fills in one
+  // accumulator), so one tile's epilogue overlaps the other pipeline's tile.
+  // Otherwise every member takes every other fill of every tile.
+  const bool pipes = !PAIR && MODE == kModeFwd && p.pipes != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -265,8 +273,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       mbar_init(full_a(s), (PAIR && rank == 0) ? kDqWarpsPerLane + 1 : kDqWarpsPerLane);
       mbar_init(a_free(s), 1);
     }
-    mbar_init(acc_full, p.n_issuers);
-    mbar_init(acc_empty, PAIR ? 8 : 4);
+    mbar_init(acc_full(0), pipes ? 1 : p.n_issuers);
+    mbar_init(acc_full(1), 1);
+    mbar_init(acc_empty(0), PAIR ? 8 : 4);
+    mbar_init(acc_empty(1), 4);
     mbar_init(drain_bar, p.n_issuers);
     *abort_flag = 0;
     fence_barrier_init();
@@ -319,15 +329,24 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       const uint32_t tx = b_bytes + kWqFill + kScFill;
       int st = pw;                           // stage of the next own fill
       uint32_t ph = 0;
-      long long f0 = 0, last_own = -1;       // first fill of the tile
-      int r0 = 0;                            // f0 % kProdWarps
+      // g: ring index of the next own fill (pw, pw + 2, ...; with tile
+      // pipelines a virtual index, since the member then takes whole tiles).
+      long long g_next = pw, last_own = -1;
+      int r0 = 0;                            // (first fill of the tile) % kProdWarps
       bool ok = true;
-      for (int t = t_first; t < total && ok; t += t_step) {
+      int li = 0;                            // this CTA's tile count
+      for (int t = t_first; t < total && ok; t += t_step, ++li) {
+        int kb0 = (pw - r0 + kProdWarps) % kProdWarps, kbs = kProdWarps;
+        r0 = (r0 + nkb) % kProdWarps;
+        if (pipes) {
+          if ((li & 1) != pw) continue;
+          kb0 = 0;
+          kbs = 1;
+        }
         const Tile tl = tile_at(t);
         // A pair's CTAs hold token rows [0, w/2) and [w/2, w) of the tile.
         const int brow = tl.row0 + static_cast<int>(rank) * (tl.width >> 1);
-        for (int kb = (pw - r0 + kProdWarps) % kProdWarps; kb < nkb; kb += kProdWarps) {
-          const long long f = f0 + kb;
+        for (int kb = kb0; kb < nkb; kb += kbs) {
           if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t bar = full_tma(st);
           mbar_arrive_expect_tx(bar, tx);
@@ -347,12 +366,11 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             tma_load_3d_hint(W_at(st), &tm_wq, bar, tl.ft * 64, tl.e * N + kb * kFillK, 0, pol_w);
             tma_load_3d_hint(S_at(st), &tm_sc, bar, kb * kFillK, tl.e * (K / 32) + tl.ft * 4, 0, pol_w);
           }
-          last_own = f;
+          last_own = g_next;
+          g_next += kProdWarps;
           st += kProdWarps;
           if (st >= S) { st -= S; ph ^= 1u; }
         }
-        f0 += nkb;
-        r0 = (r0 + nkb) % kProdWarps;
       }
       if (!ok) {
         // Let this producer's copies that may still be in flight land before
@@ -408,13 +426,22 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         if constexpr (PAIR) return mbar_wait_cluster(bar, parity, abort_flag);
         else return mbar_wait(bar, parity, abort_flag);
       };
-      for (int t = t_first; t < total && ok; t += t_step, ++it) {
+      int li = 0;                             // this CTA's tile count
+      for (int t = t_first; t < total && ok; t += t_step, ++li) {
+        int kb0 = (j - r0 + NI) % NI, kbs = NI;
+        r0 = (r0 + nkb) % NI;
+        if (pipes) {
+          if ((li & 1) != j) continue;
+          kb0 = 0;
+          kbs = 1;
+        }
+        const int q_acc = pipes ? j : 0;       // accumulator handoff barriers of this tile
         const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kTileF : kTileF, tile_at(t).width,
                                               MODE == kModeBwd ? 1u : 0u, 0u);
-        if (!wait_x(acc_empty, static_cast<uint32_t>(it & 1) ^ 1u)) { ok = false; break; }
+        if (!wait_x(acc_empty(q_acc), static_cast<uint32_t>(it & 1) ^ 1u)) { ok = false; break; }
         tc_fence_after();
         uint32_t acc = 0;
-        for (int kb = (j - r0 + NI) % NI; kb < nkb; kb += NI) {
+        for (int kb = kb0; kb < nkb; kb += kbs) {
           {
             if (!wait_x(full_a(sa), pha)) { ok = false; break; }
             tc_fence_after();
@@ -447,8 +474,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           sa += NI;
           if (sa >= SA) { sa -= SA; pha ^= 1u; }
         }
-        r0 = (r0 + nkb) % NI;
-        if (ok) commit(acc_full);             // arrives even when this issuer had no fill
+        if (ok) commit(acc_full(q_acc));      // arrives even when this issuer had no fill
+        ++it;                                 // tiles this issuer has handed over
       }
       // All MMAs of this CTA (of the pair) done before tensor memory is released.
       commit(drain_bar);
@@ -476,10 +503,16 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     int st = grp, sa = grp;                 // fill ring and A ring positions of the next own fill
     uint32_t ph = 0, pha = 0;
     bool ok = true;
-    for (int t = t_first; t < total && ok; t += t_step) {
-      const int kb_first = (grp - r0 + kLanes) % kLanes;
+    int li = 0;                             // this CTA's tile count
+    for (int t = t_first; t < total && ok; t += t_step, ++li) {
+      int kb_first = (grp - r0 + kLanes) % kLanes, kb_step = kLanes;
       r0 = (r0 + nkb) % kLanes;
-      for (int kb = kb_first; kb < nkb; kb += kLanes) {
+      if (pipes) {
+        if ((li & 1) != grp) continue;
+        kb_first = 0;
+        kb_step = 1;
+      }
+      for (int kb = kb_first; kb < nkb; kb += kb_step) {
         const int cur = st, cur_a = sa;
         const uint32_t cur_ph = ph, cur_pha = pha;
         const int kb_cur = kb;
@@ -573,18 +606,23 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     for (int t = t_first; t < total; t += t_step, ++it) {
       const Tile tl = tile_at(t);
       // Issuer j wrote its partial in this tile iff one of the tile's nkb
-      // fills f has f % NI == j.
+      // fills f has f % NI == j. With tile pipelines the tile's whole sum is
+      // in accumulator it % 2.
       const bool has0 = ((NI - r0) % NI) < nkb;
       const bool has1 = NI > 1 && ((1 + NI - r0) % NI) < nkb;
       const bool has2 = NI > 2 && ((2 + NI - r0) % NI) < nkb;
       r0 = (r0 + nkb) % NI;
+      const int q_acc = pipes ? (it & 1) : 0;
       // Tensor-memory column offsets of the written partials, in issuer order.
       const uint32_t acc = static_cast<uint32_t>(p.acc_cols);
-      const int nv = int(has0) + int(has1) + int(has2);
-      const uint32_t pc0 = has0 ? 0u : (has1 ? acc : 2 * acc);
+      const int nv = pipes ? 1 : int(has0) + int(has1) + int(has2);
+      const uint32_t pc0 = pipes ? static_cast<uint32_t>(q_acc) * acc
+                                 : (has0 ? 0u : (has1 ? acc : 2 * acc));
       const uint32_t pc1 = (has0 && has1) ? acc : 2 * acc;
       const uint32_t pc2 = 2 * acc;
-      if (!mbar_wait(acc_full, static_cast<uint32_t>(it & 1), abort_flag)) break;
+      if (!mbar_wait(acc_full(q_acc), static_cast<uint32_t>((pipes ? (it >> 1) : it) & 1),
+                     abort_flag))
+        break;
       tc_fence_after();
       const uint32_t tcol = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
       for (int c0 = 0; c0 < tl.width; c0 += 16) {
@@ -717,8 +755,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(acc_empty, 0));
-        else mbar_arrive(acc_empty);
+        if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(acc_empty(0), 0));
+        else mbar_arrive(acc_empty(q_acc));
       }
     }
   }
@@ -831,7 +869,7 @@ uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair) {
 uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E) {
   // barriers, TMEM slot + abort flag (16 B), warp totals, tile list, epilogue
   // staging (4 x 4 KiB, 128-byte aligned), alignment slack
-  return 8u * (2u * stages + 2u * a_stages + 3u) + 16u + 32u * 4u +
+  return 8u * (2u * stages + 2u * a_stages + 5u) + 16u + 32u * 4u +
          static_cast<uint32_t>(E + 1) * 4u + 128u + 4u * 4096u + 1024u;
 }
 

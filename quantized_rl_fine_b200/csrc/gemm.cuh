@@ -28,6 +28,7 @@ struct GemmArgs {
   int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages);
                               // multiple of the lane count
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
+  int32_t pipes;              // 1: two tile pipelines (two lanes, two issuers; not with pairs)
   __nv_bfloat16* out;         // [M][ldo]
   int64_t ldo;
   __nv_bfloat16* saved;       // fwd SwiGLU: written [M][N]; bwd SwiGLU: read [M][2K]

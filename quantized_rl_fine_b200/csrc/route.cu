@@ -384,6 +384,7 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
     // The tail's dynamic shared memory may pass 48 KiB: raise the limit once
     // per device (later calls, including ones under stream capture, skip it).
     static bool raised[64] = {false};
+    static int sm_count[64] = {0};
     int dev = 0;
     err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
@@ -391,6 +392,8 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
     if (!raised[dev]) {
       err = cudaFuncSetAttribute(route_tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(2 * (kTailMaxWords + 1024) * sizeof(uint32_t)));
+      if (err != cudaSuccess) return err;
+      err = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
       if (err != cudaSuccess) return err;
       raised[dev] = true;
     }
@@ -400,9 +403,7 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
     const int M = T * k;
     int blocks = 1;
     if (x != nullptr) {
-      int dev_sms = 148;
-      cudaDeviceGetAttribute(&dev_sms, cudaDevAttrMultiProcessorCount, dev);
-      blocks = std::max(1, std::min(dev_sms, (M + 7) / 8));
+      blocks = std::max(1, std::min(sm_count[dev], (M + 7) / 8));
       blocks = std::max(blocks, (M + kTailRowsPerBlock - 1) / kTailRowsPerBlock);
     } else if (M > kTailRowsPerBlock) {
       blocks = (M + kTailRowsPerBlock - 1) / kTailRowsPerBlock;

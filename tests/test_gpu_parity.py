@@ -305,3 +305,15 @@ def test_cta_pair_forward_matches_the_oracle(monkeypatch, cfg):
     monkeypatch.setenv("MOEQ_PAIR", "1")
     _run_layer_and_compare(cfg)
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, RAGGED_MX], ids=["int4", "mxfp4_ragged"])
+def test_forward_without_tile_pipelines_matches_the_oracle(monkeypatch, cfg):
+    """Two-lane forward kernels run as two tile pipelines by default (each
+    issuer accumulates whole tiles); this runs them with every issuer taking
+    every other fill of every tile instead, the layout the four-lane and the
+    one-issuer plans use."""
+    monkeypatch.setenv("MOEQ_PIPES", "0")
+    monkeypatch.setenv("MOEQ_LANES", "2")
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
