@@ -231,14 +231,15 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
     }
     pl.tmem_cols = next_pow2(pl.n_issuers * pl.acc_cols);
   }
-  // Two tile pipelines (forward; each issuer accumulates whole tiles, so one
-  // tile's epilogue overlaps the other's MMAs) need two lanes and two
-  // issuers. Measured against every issuer taking every other fill: -0.6 %
-  // (C2) to -9 % (an MXFP4 shape at 256 rows per expert), no shape slower.
+  // Two tile pipelines (each issuer accumulates whole tiles, so one tile's
+  // epilogue overlaps the other's MMAs) need two lanes and two issuers.
+  // Measured against every issuer taking every other fill: forward -0.6 %
+  // (C2) to -9 % (an MXFP4 shape at 256 rows per expert), backward -5 % to
+  // -19 % (the SwiGLU backward epilogue is the heaviest); no shape slower.
   // MOEQ_PIPES=0 turns them off (tuning only).
   pl.pipes = true;
   if (const char* env = getenv("MOEQ_PIPES")) pl.pipes = (atoi(env) != 0);
-  pl.pipes = pl.pipes && mode == kModeFwd && pl.lanes == 2 && pl.n_issuers == 2 && !pl.pair;
+  pl.pipes = pl.pipes && pl.lanes == 2 && pl.n_issuers == 2 && !pl.pair;
   const int stages = pl.stages;
   pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
   const int64_t bound = static_cast<int64_t>(pl.pair ? pl.n_ftiles / 2 : pl.n_ftiles) *

@@ -255,12 +255,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-  // Tile pipelines (forward; two lanes, two issuers, two producers): the
+  // Tile pipelines (two lanes, two issuers, two producers): the
   // CTA's i-th tile belongs to pipeline i % 2 as a whole (its producer,
   // dequant lane and issuer, which accumulates all of its fills in one
   // accumulator), so one tile's epilogue overlaps the other pipeline's tile.
   // Otherwise every member takes every other fill of every tile.
-  const bool pipes = !PAIR && MODE == kModeFwd && p.pipes != 0;
+  const bool pipes = !PAIR && p.pipes != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -610,7 +610,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       // in accumulator it % 2.
       const bool has0 = ((NI - r0) % NI) < nkb;
       const bool has1 = NI > 1 && ((1 + NI - r0) % NI) < nkb;
-      const bool has2 = NI > 2 && ((2 + NI - r0) % NI) < nkb;
+      const bool has2 = kMaxIssuers > 2 && NI > 2 && ((2 + NI - r0) % NI) < nkb;
       r0 = (r0 + nkb) % NI;
       const int q_acc = pipes ? (it & 1) : 0;
       // Tensor-memory column offsets of the written partials, in issuer order.
@@ -756,7 +756,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       __syncwarp();
       if (lane == 0) {
         if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(acc_empty(0), 0));
-        else mbar_arrive(acc_empty(q_acc));
+        else mbar_arrive(acc_empty(pipes ? (it & 1) : 0));
       }
     }
   }
