@@ -545,10 +545,8 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
   void* dxa = ws;
   st = run_gemm(kModeBwd, epi, dout, M, w, g, dxa, w->K, nullptr, pl, s);
   if (st != MOE_OK) return st;
-  cudaError_t e = launch_adapter_apply(dxa, adapter, g->expert_offsets, w->E, static_cast<int>(M),
-                                       w->K, din, true, s);
-  if (e != cudaSuccess) return MOE_ERR_CUDA;
-  return cuda_status(launch_adapter_grad(a, dxa, g->expert_offsets, w->E, w->K, d_adapter, s));
+  return cuda_status(launch_adapter_bwd(a, dxa, adapter, g->expert_offsets, w->E, w->K, din,
+                                        d_adapter, s));
 }
 
 moe_status moe_unpermute_combine(const void* rows, const int32_t* inv_perm, const float* gates,
