@@ -377,7 +377,7 @@ def _launches_per_step(cfg):
     if cfg.train:
         n += 1 + 2 + 1                          # scatter, two bwd GEMMs, unpermute-sum
         if cfg.adapter:
-            n += 2                              # adapter backward (dx, dR)
+            n += 1                              # adapter backward (dx and dR in one kernel)
     return n
 
 
