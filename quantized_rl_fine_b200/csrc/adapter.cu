@@ -195,94 +195,6 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                : "r"(addr));
 }
 
-// grid (E, ceil(K / 256)), 256 threads: dR[e][b] for the 8 column blocks b of
-// this CTA (one warp each) over the rows of expert e, 32 rows per step in
-// ascending order: the warp stages the rows' x and dx' columns of its block in
-// shared memory (rows past the expert as zeros) and forms
-// dR += x^T (32 x 32 rows) . dx' (32 rows x 32): A = x^T and B = dx' both come
-// from the staged row-major tiles through transposing matrix loads.
-__global__ void __launch_bounds__(256)
-adapter_grad_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ dxp,
-                    const int32_t* __restrict__ offsets, int K, float* __restrict__ dR) {
-  grid_dependency_wait();
-  grid_dependents_launch();
-  __shared__ __align__(16) uint16_t xs[kGradWarps][kGradRows][kStageLd];
-  __shared__ __align__(16) uint16_t gs[kGradWarps][kGradRows][kStageLd];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int e = blockIdx.x;
-  const int b = blockIdx.y * kGradWarps + warp;
-  const int nb = K / 32;
-  if (b >= nb) return;                   // warp-uniform; the warps never sync with each other
-  const int p0 = offsets[e], p1 = offsets[e + 1];
-  float acc[2][4][4];                    // [i tile][j tile][fragment]
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[mi][nt][c] = 0.0f;
-  const uint32_t xs0 = smem_u32(&xs[warp][0][0]);
-  const uint32_t gs0 = smem_u32(&gs[warp][0][0]);
-  // ldmatrix row addresses of this lane: matrix m = lane / 8, its row lane % 8.
-  const int m = lane >> 3, mr = lane & 7;
-  for (int c0 = p0; c0 < p1; c0 += kGradRows) {
-    // 32 rows x 4 chunks of 16 bytes per operand: four chunks per lane.
-    uint4 vx[4], vg[4];
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
-      const bool ok = c0 + row < p1;
-      const int64_t gi = static_cast<int64_t>(ok ? c0 + row : p0) * K + 32 * b + 8 * ch;
-      vx[h] = ok ? __ldg(reinterpret_cast<const uint4*>(x + gi)) : make_uint4(0, 0, 0, 0);
-      vg[h] = ok ? __ldg(reinterpret_cast<const uint4*>(dxp + gi)) : make_uint4(0, 0, 0, 0);
-    }
-    __syncwarp();                        // the previous step's matrix loads are done
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
-      *reinterpret_cast<uint4*>(&xs[warp][row][8 * ch]) = vx[h];
-      *reinterpret_cast<uint4*>(&gs[warp][row][8 * ch]) = vg[h];
-    }
-    __syncwarp();
-#pragma unroll
-    for (int s = 0; s < kGradRows / 16; ++s) {
-      // A = x^T (i x k): matrices (i 0-7, k 0-7), (i 8-15, k 0-7), (i 0-7, k 8-15),
-      // (i 8-15, k 8-15) of i tile mi, read from the [k][i] tile transposed.
-      uint32_t af[2][4];
-#pragma unroll
-      for (int mi = 0; mi < 2; ++mi) {
-        const int krow = 16 * s + 8 * (m >> 1) + mr;
-        const int icol = 16 * mi + 8 * (m & 1);
-        ldsm_x4_trans(xs0 + (krow * kStageLd + icol) * 2, af[mi][0], af[mi][1], af[mi][2], af[mi][3]);
-      }
-      // B = dx' (k x j): matrices (j tile nt, k 0-7), (nt, k 8-15), (nt + 1, k 0-7),
-      // (nt + 1, k 8-15), read from the [k][j] tile transposed.
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        const int krow = 16 * s + 8 * (m & 1) + mr;
-        const int jcol = 8 * (2 * np + (m >> 1));
-        uint32_t b00, b01, b10, b11;
-        ldsm_x4_trans(gs0 + (krow * kStageLd + jcol) * 2, b00, b01, b10, b11);
-#pragma unroll
-        for (int mi = 0; mi < 2; ++mi) {
-          mma16816(acc[mi][2 * np], af[mi], b00, b01);
-          mma16816(acc[mi][2 * np + 1], af[mi], b10, b11);
-        }
-      }
-    }
-  }
-  float* dst = dR + (static_cast<int64_t>(e) * nb + b) * 1024;
-#pragma unroll
-  for (int mi = 0; mi < 2; ++mi)
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int i = 16 * mi + g, j = 8 * nt + 2 * t;
-      *reinterpret_cast<float2*>(dst + i * 32 + j) = make_float2(acc[mi][nt][0], acc[mi][nt][1]);
-      *reinterpret_cast<float2*>(dst + (i + 8) * 32 + j) = make_float2(acc[mi][nt][2], acc[mi][nt][3]);
-    }
-}
-
 // Backward, fused: grid (E, ceil(K / 256)), 256 threads. Warp (e, b) walks the
 // rows of expert e in ascending order, 32 at a time: it stages the rows' x and
 // dx' columns of block b in shared memory and from them forms both
@@ -411,17 +323,15 @@ adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
 }  // namespace
 
 cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* offsets, int E,
-                                 int M, int K, void* out, bool transpose, cudaStream_t s) {
+                                 int M, int K, void* out, cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int nb = K / 32;
   const int64_t spans = (static_cast<int64_t>(M) + 16 * kApplyGroups - 1) / (16 * kApplyGroups);
   const int64_t ctas = (spans * nb + 7) / 8;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(ctas));
-  return launch_pdl(transpose ? adapter_apply_kernel<1> : adapter_apply_kernel<0>, grid, dim3(256),
-                    0, s, static_cast<const __nv_bfloat16*>(x),
-                    static_cast<const __nv_bfloat16*>(R), offsets, E, M, K,
-                    static_cast<__nv_bfloat16*>(out));
+  return launch_pdl(adapter_apply_kernel<0>, dim3(static_cast<unsigned>(ctas)), dim3(256), 0, s,
+                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(R),
+                    offsets, E, M, K, static_cast<__nv_bfloat16*>(out));
 }
 
 cudaError_t launch_adapter_bwd(const void* x, const void* dxp, const void* R,
@@ -433,15 +343,6 @@ cudaError_t launch_adapter_bwd(const void* x, const void* dxp, const void* R,
                     static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dxp),
                     static_cast<const __nv_bfloat16*>(R), offsets, K,
                     static_cast<__nv_bfloat16*>(dx), dR);
-}
-
-cudaError_t launch_adapter_grad(const void* x, const void* dxp, const int32_t* offsets, int E,
-                                int K, float* dR, cudaStream_t s) {
-  const int nb = K / 32;
-  dim3 grid(E, (nb + kGradWarps - 1) / kGradWarps);
-  return launch_pdl(adapter_grad_kernel, grid, dim3(256), 0, s,
-                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dxp),
-                    offsets, K, dR);
 }
 
 }  // namespace moeq

@@ -505,7 +505,7 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
   if (adapter) {
     void* xa = ws;
     cudaError_t e = launch_adapter_apply(a, adapter, g->expert_offsets, w->E, static_cast<int>(M),
-                                         w->K, xa, false, s);
+                                         w->K, xa, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     bmat = xa;
   }

@@ -14,14 +14,13 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                          void* x_perm, int32_t* block_counts, cudaStream_t s);
 cudaError_t launch_combine(const void* rows, const int32_t* inv_perm, const float* gates, int T,
                            int k, int64_t D, void* out, int mode, cudaStream_t s);
+// out = x . R_e for the rows of each expert (forward adapter).
 cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* offsets, int E,
-                                 int M, int K, void* out, bool transpose, cudaStream_t s);
+                                 int M, int K, void* out, cudaStream_t s);
 // dx = dxp . R_e^T and dR = sum over each expert's rows of x^T dxp, in one pass.
 cudaError_t launch_adapter_bwd(const void* x, const void* dxp, const void* R,
                                const int32_t* offsets, int E, int K, void* dx, float* dR,
                                cudaStream_t s);
-cudaError_t launch_adapter_grad(const void* x, const void* dxp, const int32_t* offsets, int E,
-                                int K, float* dR, cudaStream_t s);
 cudaError_t launch_dequant_rows(const void* packed, const void* scales, int64_t R, int K, int fmt,
                                 void* out, cudaStream_t s);
 
