@@ -50,6 +50,12 @@ __device__ __forceinline__ int expert_of_row(const int32_t* offsets, int E, int 
   return lo;
 }
 
+// The same for a row at or after one whose expert e is known: step forward.
+__device__ __forceinline__ int expert_of_row_from(const int32_t* offsets, int E, int e, int row) {
+  while (e + 1 < E && __ldg(offsets + e + 1) <= row) ++e;
+  return e;
+}
+
 constexpr int kApplyGroups = 4;   // 16-row groups per warp task of the apply kernel
 constexpr int kStageLd = 40;      // staged row length in BF16 (80 bytes: conflict-free ldmatrix)
 
@@ -130,6 +136,8 @@ adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
   const uint32_t tl0 = smem_u32(&tl[0][0]);
   const int m = lane >> 3, mr = lane & 7;   // ldmatrix: matrix m, its row mr
   int cached = -1;
+  // Expert of the task's first row (one search); the groups step forward from it.
+  int e_run = expert_of_row(offsets, E, span0);
   uint32_t bf[4][2][2];
   for (int q = 0; q < kApplyGroups; ++q) {
     const int r0 = span0 + 16 * q;
@@ -142,8 +150,9 @@ adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
       ldsm_x4(tl0 + (row * kStageLd + col) * 2, a[s][0], a[s][1], a[s][2], a[s][3]);
     }
     const int ra = r0 + g, rb = ra + 8;
-    const int e_first = expert_of_row(offsets, E, r0);
-    const int e_last = expert_of_row(offsets, E, min(r0 + 15, M - 1));
+    const int e_first = expert_of_row_from(offsets, E, e_run, r0);
+    const int e_last = expert_of_row_from(offsets, E, e_first, min(r0 + 15, M - 1));
+    e_run = e_last;
     float res[4][4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
