@@ -260,7 +260,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   // dequant lane and issuer, which accumulates all of its fills in one
   // accumulator), so one tile's epilogue overlaps the other pipeline's tile.
   // Otherwise every member takes every other fill of every tile.
-  const bool pipes = !PAIR && p.pipes != 0;
+  // (Only with exactly two lanes and two issuers: the planner asks for it
+  // only then, and any other layout would leave a member without tiles.)
+  const bool pipes = !PAIR && LANES == 2 && p.n_issuers == 2 && p.pipes != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
