@@ -17,8 +17,9 @@
  * quantized weights fine-tuned directly without storing a dequantized base);
  * open-weight MoE explainer, section 3 (MXFP4: 4-bit elements in groups of 32
  * with one shared scale). Here no dequantized weight is ever written to
- * global memory: each kernel dequantizes a tile into shared memory and feeds
- * the tensor cores from there.
+ * global memory: each GEMM kernel dequantizes a tile into tensor memory
+ * (forward) or shared memory (backward) and feeds the tensor cores from
+ * there.
  *
  * Conventions for every entry point
  *  - All tensor pointers are DEVICE pointers, allocated and owned by the
@@ -134,7 +135,9 @@ typedef struct moe_groups {
  *              then ascending token id.
  *  inv_perm    [T*k] int32: permuted row of (token t, slot j) at t*k + j.
  *  x_perm      [T*k][d] bf16: x_perm[p] = x[perm_token[p]] (bit copy).
- *  ws          scratch of the per-block expert histograms.
+ *  ws          scratch of the per-block expert histograms (used by launches
+ *              beyond the single-pass tail, T > 1024 or E*ceil(T/32) > 8192;
+ *              the size query covers every case).
  * Requires T >= 1, 1 <= E <= 1024, d % 8 == 0 when x is given,
  * T*k < 2^31.
  */
