@@ -126,3 +126,26 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         moeq.moe_route_permute(torch.zeros((4, 4)), None, 2, 1)
+
+
+def test_plain_c_host_compiles_links_and_calls(L, tmp_path):
+    """The header is plain C99 (no CUDA or C++ headers needed), and a C program
+    links against the library and calls the host-only entry points."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler on this host")
+    src = tmp_path / "host.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "moeq.h"\n'
+        "int main(void) {\n"
+        '  printf("%d %s\\n", (int)moe_abi_version(), moe_status_string(MOE_ERR_WORKSPACE));\n'
+        "  return 0;\n}\n")
+    exe = tmp_path / "host"
+    libdir = os.path.dirname(moeq.LIB_PATH)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lmoeq", "-Wl,-rpath," + libdir],
+                   check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == [str(L.moe_abi_version()), "MOE_ERR_WORKSPACE"]
