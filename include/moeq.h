@@ -55,7 +55,11 @@
  *    w = bf16(e2m1 * 2^(X-127)), exact except overflow to inf.
  *  Requirements: K % 64 == 0, N % 64 == 0 (N % 128 == 0 for the SwiGLU
  *  gate/up weight, whose rows 0..N/2-1 are the gate and N/2..N-1 the up
- *  projection), 1 <= E <= 1024, E*N < 2^31.
+ *  projection), 1 <= E <= 1024, E*N < 2^31. Other shapes return
+ *  MOE_ERR_UNSUPPORTED without launching. (The kernels stream the reduction
+ *  in 64-element halves of 128-wide steps and write output features in
+ *  blocks of 32 or 64; every expert shape of the Orbit and MXFP4 pages is a
+ *  multiple of 512.)
  */
 #ifndef MOEQ_H
 #define MOEQ_H
@@ -135,9 +139,11 @@ typedef struct moe_groups {
  *              then ascending token id.
  *  inv_perm    [T*k] int32: permuted row of (token t, slot j) at t*k + j.
  *  x_perm      [T*k][d] bf16: x_perm[p] = x[perm_token[p]] (bit copy).
- *  ws          scratch of the per-block expert histograms (used by launches
- *              beyond the single-pass tail, T > 1024 or E*ceil(T/32) > 8192;
- *              the size query covers every case).
+ *  ws          scratch of the per-block expert histograms. Launches that
+ *              take the single-pass tail (T <= 1024 and E*ceil(T/32) <= 8192)
+ *              need none: the size query returns 0 and (ws, ws_bytes) may both
+ *              be NULL. Larger launches need ceil(T/64)*E int32 (rounded up to
+ *              256 bytes).
  * Requires T >= 1, 1 <= E <= 1024, d % 8 == 0 when x is given,
  * T*k < 2^31.
  */
@@ -165,13 +171,17 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
  * ceil(T/64) * E > 2^20, are rejected with MOE_ERR_WORKSPACE before anything
  * is launched. The call itself never allocates or frees device memory.
  *
- * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture. All calls on a device share the one array: calls whose kernels
- * overlap on the GPU (different streams without ordering between them) race
- * on it and give wrong results. Calls ordered on one stream are safe; each
- * call rewrites the entries it reads, so leftovers of an earlier call do not
- * matter.
+ * The first call on a device does this library's one-time setup there: it
+ * looks up the array's device address (with that device current) and caches
+ * it, and it sets the routing kernels' shared-memory limit. Make that first
+ * call before any stream capture; later calls do no setup. The cached
+ * address belongs to the device's current context: after cudaDeviceReset the
+ * array may live elsewhere, so do not call this entry point again in that
+ * process after a reset. All calls on a device share the one array: calls
+ * whose kernels overlap on the GPU (different streams without ordering
+ * between them) race on it and give wrong results. Calls ordered on one
+ * stream are safe; each call rewrites the entries it reads, so leftovers of
+ * an earlier call do not matter.
  */
 moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t T, int32_t E,
                                      int32_t k, int64_t d, int32_t chunk_size, int32_t* topk_idx,

@@ -382,11 +382,14 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
   if (T < 1 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || chunk_size < 1)
     return MOE_ERR_INVALID_ARG;
   if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
-  const int nblk = route_num_blocks(T);
-  const size_t need = align_up(static_cast<size_t>(nblk) * E * sizeof(int32_t), 256);
+  // Launches that take the single-pass tail need no scratch (size 0); larger
+  // ones keep per-block expert histograms in the workspace.
+  const size_t need = route_single_pass(T, E)
+                          ? 0
+                          : align_up(static_cast<size_t>(route_num_blocks(T)) * E * sizeof(int32_t), 256);
   moe_status st = check_workspace(ws, ws_bytes, need);
   if (st != MOE_OK) return st;
-  if (!ws) return MOE_OK;   // size query
+  if (!ws && ws_bytes) return MOE_OK;   // size query
   const void* ptrs[] = {logits, topk_idx, gates, expert_offsets, active, num_active,
                         chunk_offsets, num_chunks, perm_token, inv_perm};
   for (const void* p : ptrs) {
@@ -439,6 +442,9 @@ moe_status static_scratch_on_current_device(int32_t** out) {
   if (!g_static_scratch_addr[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_static_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    // The routing kernels' own one-time setup on this device, done here too,
+    // so that after the first call no later call does any setup.
+    if (route_prepare_device(nullptr) != cudaSuccess) return MOE_ERR_CUDA;
     g_static_scratch_addr[dev] = static_cast<int32_t*>(p);
   }
   *out = g_static_scratch_addr[dev];

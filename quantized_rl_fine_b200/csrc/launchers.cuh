@@ -7,6 +7,12 @@
 namespace moeq {
 
 int route_num_blocks(int64_t T);
+// True when a routing launch takes the single-pass tail (no per-block
+// histograms, so no scratch memory).
+bool route_single_pass(int64_t T, int E);
+// One-time per-device setup of the routing kernels (thread-safe); writes the
+// device's SM count when sm_count is not NULL.
+cudaError_t route_prepare_device(int* sm_count);
 cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k, int64_t d,
                          int chunk_size, int32_t* topk_idx, float* gates, int32_t* offsets,
                          int32_t* active, int32_t* num_active, int32_t* chunk_offsets,

@@ -25,6 +25,7 @@
 // offsets and stable ranks from popcounts of those masks; the serial walk
 // over the per-block histograms, and one launch, go away.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "launchers.cuh"
@@ -354,6 +355,41 @@ int route_num_blocks(int64_t T) {
   return static_cast<int>((T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock);
 }
 
+bool route_single_pass(int64_t T, int E) {
+  const int64_t W = (T + 31) / 32;
+  return W <= 32 && W * E <= kTailMaxWords;
+}
+
+namespace {
+
+std::mutex g_route_setup_mutex;
+bool g_route_setup_done[64] = {false};
+int g_route_sm_count[64] = {0};
+
+}  // namespace
+
+// The tail's dynamic shared memory may pass 48 KiB: its limit is raised once
+// per device, and the SM count read once, under a lock (so concurrent host
+// threads are safe); later calls only read the cached values, so calls made
+// during stream capture do no setup once a call on that device has run.
+cudaError_t route_prepare_device(int* sm_count) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_route_setup_mutex);
+  if (!g_route_setup_done[dev]) {
+    err = cudaFuncSetAttribute(route_tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(2 * (kTailMaxWords + 1024) * sizeof(uint32_t)));
+    if (err != cudaSuccess) return err;
+    err = cudaDeviceGetAttribute(&g_route_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return err;
+    g_route_setup_done[dev] = true;
+  }
+  if (sm_count) *sm_count = g_route_sm_count[dev];
+  return cudaSuccess;
+}
+
 cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k, int64_t d,
                          int chunk_size, int32_t* topk_idx, float* gates, int32_t* offsets,
                          int32_t* active, int32_t* num_active, int32_t* chunk_offsets,
@@ -361,7 +397,8 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                          void* x_perm, int32_t* block_counts, cudaStream_t s) {
   const int W = (T + 31) / 32;
   // Small launches: one token per warp, then the single-block tail.
-  const bool small = W <= 32 && W * E <= kTailMaxWords;
+  const bool small = route_single_pass(T, E);
+  if (!small && block_counts == nullptr) return cudaErrorInvalidValue;
   const int tpb = small ? kTopkThreads / 32 : kRouteTokensPerBlock;
   const int nblk = small ? (T + tpb - 1) / tpb : route_num_blocks(T);
   int32_t* hist_out = small ? nullptr : block_counts;
@@ -381,29 +418,16 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
 #undef MOEQ_TOPK
   if (err != cudaSuccess) return err;
   if (small) {
-    // The tail's dynamic shared memory may pass 48 KiB: raise the limit once
-    // per device (later calls, including ones under stream capture, skip it).
-    static bool raised[64] = {false};
-    static int sm_count[64] = {0};
-    int dev = 0;
-    err = cudaGetDevice(&dev);
+    int sm_count = 0;
+    err = route_prepare_device(&sm_count);
     if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!raised[dev]) {
-      err = cudaFuncSetAttribute(route_tail_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(2 * (kTailMaxWords + 1024) * sizeof(uint32_t)));
-      if (err != cudaSuccess) return err;
-      err = cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
-      if (err != cudaSuccess) return err;
-      raised[dev] = true;
-    }
     const size_t tsm = 2 * static_cast<size_t>(W + 1) * E * sizeof(uint32_t);
     // With x, one block per SM (at least enough for kTailRowsPerBlock rows
     // each) shares the row copy; without it one block does the tail alone.
     const int M = T * k;
     int blocks = 1;
     if (x != nullptr) {
-      blocks = std::max(1, std::min(sm_count[dev], (M + 7) / 8));
+      blocks = std::max(1, std::min(sm_count, (M + 7) / 8));
       blocks = std::max(blocks, (M + kTailRowsPerBlock - 1) / kTailRowsPerBlock);
     } else if (M > kTailRowsPerBlock) {
       blocks = (M + kTailRowsPerBlock - 1) / kTailRowsPerBlock;

@@ -65,8 +65,14 @@ def test_fwd_workspace_query_and_validation(L):
     assert _fwd(L, adapter=0xA0000, wsb=wsb2) == moeq.MOE_OK
     base = wsb2.value
     assert base >= 64 * 512 * 2 and base % 256 == 0                  # a' rows
+    # Shape rules (a reading of the boundary): K % 64, N % 64, and N % 128
+    # for the SwiGLU gate/up weight; a K with a 64-element tail is accepted.
     assert _fwd(L, qw=_qw(K=96)) == 3                                # K % 64
+    assert _fwd(L, qw=_qw(K=32)) == 3
     assert _fwd(L, qw=_qw(N=100)) == 3                               # N % 64
+    assert _fwd(L, qw=_qw(N=80)) == 3
+    assert _fwd(L, qw=_qw(K=576)) == moeq.MOE_OK                     # K % 128 == 64
+    assert _fwd(L, qw=_qw(N=320)) == moeq.MOE_OK                     # N % 128 == 64, no SwiGLU
     assert _fwd(L, qw=_qw(fmt=7)) == 1
     assert _fwd(L, qw=_qw(packed=0x10008)) == 2                      # misaligned
     assert _fwd(L, epi=2) == 1                                       # backward epilogue in fwd
@@ -110,7 +116,20 @@ def test_route_and_combine_validation(L):
     def route(T=64, E=8, k=2, d=256, C=8, x=p, ws=None, wsb=wsb, logits=p):
         return L.moe_route_permute(logits, x, T, E, k, d, C, p, p, p, p, p, p, p, p, p, p, ws,
                                    ctypes.byref(wsb), None)
-    assert route() == moeq.MOE_OK and wsb.value >= 8 * 4
+    # The single-pass tail (T <= 1024 and E * ceil(T/32) <= 8192) needs no
+    # workspace; larger launches need ceil(T/64) * E int32 histogram entries.
+    assert route() == moeq.MOE_OK and wsb.value == 0
+    assert route(T=1024, E=256) == moeq.MOE_OK and wsb.value == 0
+    assert route(T=1024, E=257) == moeq.MOE_OK and wsb.value >= 16 * 257 * 4
+    assert route(T=4096, E=384) == moeq.MOE_OK and wsb.value >= 64 * 384 * 4
+    assert wsb.value % 256 == 0
+    # a single-pass launch runs without any workspace (ws and ws_bytes NULL)
+    # as far as validation goes: here its misaligned logits are refused
+    assert L.moe_route_permute(p + 4, p, 64, 8, 2, 256, 8, p, p, p, p, p, p, p, p, p, p, None,
+                               None, None) == 2
+    # a larger one without a workspace is a workspace error
+    assert L.moe_route_permute(p, p, 4096, 384, 8, 256, 8, p, p, p, p, p, p, p, p, p, p, None,
+                               None, None) == 4
     assert route(k=9) == 1 and route(k=0) == 1 and route(E=1025) == 1 and route(C=0) == 1
     assert route(k=33, E=64) == 1
     full = ctypes.c_size_t(wsb.value)

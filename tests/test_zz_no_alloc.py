@@ -7,9 +7,12 @@ or a C host without a caching allocator, for which a cudaMalloc/cudaFree pair
 per call would synchronize the device. This entry point keeps its histogram
 scratch in a fixed array inside the library instead.
 
-The test calls it through the C ABI twice in a row (a larger problem, then a
-smaller one, so leftovers of the first call sit in the shared array) and
-checks every output against moe_route_permute, which uses a caller workspace.
+The test calls it through the C ABI twice in a row and checks every output
+against moe_route_permute, which uses a caller workspace. Both problems are
+large enough for the histogram path (more than 1024 tokens), which is the one
+that uses the fixed array: the first fills 47 x 384 histogram entries, the
+second reads 32 x 128 of them back after rewriting them, so it runs over the
+first call's leftovers.
 """
 
 import ctypes
@@ -44,7 +47,7 @@ def _noalloc(logits, x, k, chunk_size):
 
 
 def test_noalloc_routing_matches_workspace_routing_twice_in_a_row():
-    cases = [(3000, 384, 8, 16, 11), (777, 64, 4, 8, 12)]      # larger first, then smaller
+    cases = [(3000, 384, 8, 16, 11), (2048, 128, 4, 8, 12)]    # larger first, then smaller
     for T, E, k, C, seed in cases:
         g = torch.Generator().manual_seed(seed)
         logits = torch.randn((T, E), generator=g)
@@ -58,7 +61,7 @@ def test_noalloc_routing_matches_workspace_routing_twice_in_a_row():
         nch = int(want.num_chunks.item())
         assert int(got.num_active.item()) == A and int(got.num_chunks.item()) == nch
         assert torch.equal(got.topk_idx, want.topk_idx)
-        assert torch.allclose(got.gates, want.gates, rtol=2e-6, atol=1e-7)
+        assert torch.equal(got.gates, want.gates)                # same top-k kernel
         assert torch.equal(got.expert_offsets, want.expert_offsets)
         assert torch.equal(got.active[:A], want.active[:A])
         assert torch.equal(got.chunk_offsets[: nch + 1], want.chunk_offsets[: nch + 1])
