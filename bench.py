@@ -51,6 +51,8 @@ def _args():
     ap.add_argument("--workload", default="trillion_int4_T16384")
     ap.add_argument("--chunk", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prior-art", action="store_true",
+                    help="time the temporary-buffer scheme against the fused GEMMs, per chunk size")
     return ap.parse_args()
 
 
@@ -68,6 +70,13 @@ def _workloads():
     # expert) with 48 experts: small enough for a full ncu capture.
     w["trillion_int4_E48_T16"] = C.TRILLION_INT4.with_(
         E=48, T=16, name="trillion_int4_E48_k8_d7168_f2048_T16")
+    # The per-expert shape of the T=16384 layer (about 341 token rows per
+    # expert) and of the training step (about 85) with 48 experts: the same
+    # kernels and tiles, small enough for a full ncu capture.
+    w["trillion_int4_E48_T2048"] = C.TRILLION_INT4.with_(
+        E=48, T=2048, name="trillion_int4_E48_k8_d7168_f2048_T2048")
+    w["train_int4_E48_T512"] = C.TRAIN_INT4.with_(
+        E=48, T=512, name="train_int4_adapter_E48_k8_d7168_f2048_T512")
     return w
 
 
@@ -650,9 +659,70 @@ def run_ours(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- prior-art comparator
+
+def run_prior_art(args, cfg):
+    """One JSON line per chunk size C: the Orbit article's temporary-buffer
+    scheme (chunk of C experts dequantized to BF16, cuBLAS GEMMs, buffer
+    released) against this library's fused GEMMs on the same routed rows, with
+    the temporary memory each needs. Eager launches, CUDA events, median of
+    the repetitions; the weights (GBs) are far larger than L2."""
+    import torch
+    from quantized_rl_fine_b200 import moeq, prior_art, synth
+    from quantized_rl_fine_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = synth.make_workload(cfg, dev)
+    w_first = wl["w_gu"] if cfg.swiglu else wl["w_up"]
+    reps = max(3, min(args.steps, 10))
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps + 1):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts[1:])
+
+    for C in (8, 16, 32):
+        r = moeq.moe_route_permute(wl["logits"], wl["x"], cfg.k, C)
+        M = r.x_perm.shape[0]
+        h = torch.empty((M, cfg.f), dtype=torch.bfloat16, device=dev)
+        y = torch.empty((M, cfg.d if cfg.swiglu else cfg.f), dtype=torch.bfloat16, device=dev)
+
+        def fused():
+            if cfg.swiglu:
+                moeq.moe_grouped_qgemm_fwd(r.x_perm, w_first, r, moeq.EPI_SWIGLU, out=h)
+                moeq.moe_grouped_qgemm_fwd(h, wl["w_d"], r, moeq.EPI_NONE, out=y)
+            else:
+                moeq.moe_grouped_qgemm_fwd(r.x_perm, w_first, r, moeq.EPI_NONE, out=y)
+        got = {}
+
+        def prior():
+            got["y"], got["peak"] = prior_art.forward(r.x_perm, r, w_first, wl.get("w_d"), C,
+                                                      swiglu=cfg.swiglu)
+        t_fused = timed(fused)
+        t_prior = timed(prior)
+        diff = (got["y"].float() - y.float()).abs().max().item()
+        print(json.dumps({
+            "comparator": "temporary BF16 buffer per chunk of active experts + cuBLAS GEMMs",
+            "workload": cfg.name, "chunk_size": C, "reps": reps,
+            "prior_art_ms": t_prior, "fused_ms": t_fused, "fused_speedup": t_prior / t_fused,
+            "prior_art_peak_temp_bytes": got["peak"], "fused_temp_bytes": 0,
+            "max_abs_diff_of_per_slot_outputs": diff}), flush=True)
+        del got
+
+
 def main():
     args = _args()
     cfg = _workloads()[args.workload]
+    if args.prior_art:
+        run_prior_art(args, cfg)
+        return
     if args.impl == "reference":
         run_reference(args, cfg)
     else:

@@ -252,6 +252,56 @@ moe_status moe_unpermute_combine(const void* rows, const int32_t* inv_perm, cons
                                  int64_t T, int32_t k, int64_t D, void* out, int32_t mode,
                                  void* stream);
 
+/*
+ * moe_dequant_experts -- whole experts of a 4-bit stack dequantized into a
+ * BF16 buffer: out[i] = W[experts[i]] ([N][K] bf16, row-major) for i < count.
+ * This is the step the Orbit article's own scheme runs on each chunk of active
+ * experts ("Active-expert-chunked dequantization": the selected experts'
+ * weights are dequantized into a temporary high-precision buffer before the
+ * grouped GEMM, and the buffer is released after it). The grouped GEMMs of
+ * this library never call it; it serves the comparison with that scheme.
+ *
+ *  experts  device int32 [count], expert ids in [0, E). An id outside that
+ *           range gives zeros and sets MOE_DEVERR_BAD_OFFSETS.
+ *  out      device bf16 [count][N][K], caller-allocated (count*N*K*2 bytes).
+ * Same dequantization as the GEMM kernels, bit for bit. count == 0 launches
+ * nothing.
+ */
+moe_status moe_dequant_experts(const moe_qweight* w, const int32_t* experts, int32_t count,
+                               void* out, void* stream);
+
+/*
+ * moe_ep_regroup -- expert parallelism over W ranks: reorders the rows one
+ * rank received from its peers. The experts are split into W contiguous
+ * ranges of E_loc (rank r owns experts r*E_loc .. (r+1)*E_loc-1); every rank
+ * routes its own tokens, and the run of its x_perm rows that belongs to rank
+ * r's experts goes to rank r in one all-to-all exchange. The pages' setting
+ * (Orbit article: a trillion-parameter INT4 MoE trained in one 8xB200 node)
+ * needs this split: its base weights do not fit one GPU.
+ *
+ *  counts     device int32 [W][E_loc]: rows received from source rank s for
+ *             local expert e. The received rows are source-major: for s =
+ *             0..W-1, for e = 0..E_loc-1, the source's rows of e in its order.
+ *  R          total rows (the sum of counts, which the exchange needs on the
+ *             host anyway). A mismatch sets MOE_DEVERR_BAD_OFFSETS and copies
+ *             nothing.
+ *  rows_in, rows_out  device bf16 [R][D], D % 8 == 0.
+ *  direction  0: rows_out = rows_in reordered to local expert-major order
+ *             (expert, then source, then the source's order), and the local
+ *             group tables are written for the local grouped GEMMs:
+ *             expert_offsets [E_loc+1], active [E_loc], num_active [1],
+ *             chunk_offsets [E_loc+1], num_chunks [1] (as moe_route_permute
+ *             writes them, with chunk_size experts per chunk).
+ *             1: the inverse (local expert-major -> source-major, to send the
+ *             results back); the table pointers are not used and may be NULL.
+ * Requires 1 <= W, 1 <= E_loc, W*E_loc <= 2048.
+ */
+moe_status moe_ep_regroup(const int32_t* counts, int32_t W, int32_t E_loc, int64_t R,
+                          const void* rows_in, void* rows_out, int64_t D, int32_t direction,
+                          int32_t chunk_size, int32_t* expert_offsets, int32_t* active,
+                          int32_t* num_active, int32_t* chunk_offsets, int32_t* num_chunks,
+                          void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word of the
  * current device (MOE_DEVERR_*). Debug/test use. */
 moe_status moe_get_device_error(int32_t* code, void* stream);

@@ -43,6 +43,44 @@ __global__ void dequant_rows_kernel(const uint8_t* __restrict__ packed, const vo
   for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
 }
 
+// One thread per (listed expert, row, group): the 32 elements of one
+// quantization group of one weight row, written as 64 contiguous bytes. The
+// temporary-buffer scheme of the Orbit article dequantizes whole experts like
+// this; the grouped GEMMs of this library never do.
+template <int FMT>
+__global__ void dequant_experts_kernel(const uint8_t* __restrict__ packed,
+                                       const void* __restrict__ scales,
+                                       const int32_t* __restrict__ experts, int count, int E, int N,
+                                       int K, uint16_t* __restrict__ out) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  const int G = K / 32;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t per_expert = static_cast<int64_t>(N) * G;
+  if (gid >= per_expert * count) return;
+  const int i = static_cast<int>(gid / per_expert);
+  const int64_t rg = gid - i * per_expert;
+  const int n = static_cast<int>(rg / G);
+  const int g = static_cast<int>(rg - static_cast<int64_t>(n) * G);
+  const int e = experts[i];
+  uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<int64_t>(i) * N + n) * K + g * 32);
+  if (e < 0 || e >= E) {   // not an expert of the stack: zeros, and the error word
+    if (rg == 0) raise_device_error(MOE_DEVERR_BAD_OFFSETS);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const uint4 pk = *reinterpret_cast<const uint4*>(
+      packed + (static_cast<int64_t>(e) * N + n) * (K / 2) + g * 16);
+  const int64_t soff = (static_cast<int64_t>(e) * G + g) * N + n;
+  const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? static_cast<const uint16_t*>(scales)[soff]
+                                                      : static_cast<const uint8_t*>(scales)[soff];
+  uint32_t o[16];
+  dequant32<FMT>(pk, sbits, o);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+}
+
 // --------------------------------------------------------------- host helpers
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -586,6 +624,53 @@ moe_status moe_test_dequant(const void* packed, const void* scales, int64_t R, i
   if (!aligned16(packed) || !aligned16(scales) || !aligned16(out)) return MOE_ERR_MISALIGNED;
   return cuda_status(launch_dequant_rows(packed, scales, R, K, fmt, out,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_dequant_experts(const moe_qweight* w, const int32_t* experts, int32_t count,
+                               void* out, void* stream) {
+  moe_status st = check_qweight(w);
+  if (st != MOE_OK) return st;
+  if (!experts || !out || count < 0) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(experts) || !aligned16(out)) return MOE_ERR_MISALIGNED;
+  if (count == 0) return MOE_OK;
+  const int64_t n = static_cast<int64_t>(count) * w->N * (w->K / 32);
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  if (blocks >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint8_t* packed = static_cast<const uint8_t*>(w->packed);
+  uint16_t* o = static_cast<uint16_t*>(out);
+  cudaError_t e;
+  if (w->fmt == MOE_W_INT4_G32_BF16)
+    e = launch_pdl(dequant_experts_kernel<MOE_W_INT4_G32_BF16>, dim3(static_cast<unsigned>(blocks)),
+                   dim3(threads), 0, s, packed, w->scales, experts, count, w->E, w->N, w->K, o);
+  else
+    e = launch_pdl(dequant_experts_kernel<MOE_W_MXFP4_G32_E8M0>, dim3(static_cast<unsigned>(blocks)),
+                   dim3(threads), 0, s, packed, w->scales, experts, count, w->E, w->N, w->K, o);
+  return cuda_status(e);
+}
+
+moe_status moe_ep_regroup(const int32_t* counts, int32_t W, int32_t E_loc, int64_t R,
+                          const void* rows_in, void* rows_out, int64_t D, int32_t direction,
+                          int32_t chunk_size, int32_t* expert_offsets, int32_t* active,
+                          int32_t* num_active, int32_t* chunk_offsets, int32_t* num_chunks,
+                          void* stream) {
+  if (!counts || W < 1 || E_loc < 1 || static_cast<int64_t>(W) * E_loc > ep_max_entries())
+    return MOE_ERR_INVALID_ARG;
+  if (R < 0 || R >= (int64_t(1) << 31) || D < 8 || D % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (direction != 0 && direction != 1) return MOE_ERR_INVALID_ARG;
+  if (R > 0 && (!rows_in || !rows_out)) return MOE_ERR_INVALID_ARG;
+  if (direction == 0 && (chunk_size < 1 || !expert_offsets || !active || !num_active ||
+                         !chunk_offsets || !num_chunks))
+    return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {counts, rows_in, rows_out, expert_offsets, active, num_active,
+                        chunk_offsets, num_chunks};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_ep_regroup(counts, W, E_loc, static_cast<int>(R), rows_in, rows_out, D,
+                                       direction, chunk_size, expert_offsets, active, num_active,
+                                       chunk_offsets, num_chunks, num_sms(),
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_test_set_wait_budget(int64_t cycles) {

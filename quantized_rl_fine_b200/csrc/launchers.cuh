@@ -27,6 +27,13 @@ cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* of
 cudaError_t launch_adapter_bwd(const void* x, const void* dxp, const void* R,
                                const int32_t* offsets, int E, int K, void* dx, float* dR,
                                cudaStream_t s);
+// Expert parallelism: received rows, source-major <-> local expert-major
+// (dir 0 / 1); dir 0 also writes the local group tables.
+cudaError_t launch_ep_regroup(const int32_t* counts, int W, int E_loc, int R, const void* in,
+                              void* out, int64_t D, int dir, int chunk_size, int32_t* offsets,
+                              int32_t* active, int32_t* num_active, int32_t* chunk_offsets,
+                              int32_t* num_chunks, int sm_count, cudaStream_t s);
+int ep_max_entries();
 cudaError_t launch_dequant_rows(const void* packed, const void* scales, int64_t R, int K, int fmt,
                                 void* out, cudaStream_t s);
 

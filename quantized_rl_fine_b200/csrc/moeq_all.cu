@@ -4,5 +4,6 @@
 #include "api.cu"
 #include "adapter.cu"
 #include "combine.cu"
+#include "ep.cu"
 #include "gemm.cu"
 #include "route.cu"

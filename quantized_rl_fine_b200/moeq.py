@@ -31,7 +31,8 @@ DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_OFFSETS = 0, 1, 2
 
 EXPORTED = ("moe_route_permute", "moe_route_permute_noalloc", "moe_grouped_qgemm_fwd", "moe_grouped_qgemm_bwd_dx",
             "moe_unpermute_combine", "moe_get_device_error", "moe_status_string",
-            "moe_abi_version", "moe_test_dequant", "moe_test_set_wait_budget")
+            "moe_abi_version", "moe_test_dequant", "moe_test_set_wait_budget",
+            "moe_dequant_experts", "moe_ep_regroup")
 
 
 class MoeError(RuntimeError):
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.moe_abi_version.argtypes = []
     L.moe_test_dequant.argtypes = [vp, vp, i64, i32, i32, vp, vp]
     L.moe_test_set_wait_budget.argtypes = [i64]
+    L.moe_dequant_experts.argtypes = [ctypes.POINTER(QWeightC), vp, i32, vp, vp]
+    L.moe_ep_regroup.argtypes = [vp, i32, i32, i64, vp, vp, i64, i32, i32, vp, vp, vp, vp, vp, vp]
     for name in EXPORTED:
         if name not in ("moe_status_string",):
             getattr(L, name).restype = ctypes.c_int32
@@ -260,6 +263,48 @@ def moe_test_dequant(packed: torch.Tensor, scales: torch.Tensor, fmt: str, strea
     _check(lib().moe_test_dequant(_p(packed), _p(scales), R, 2 * half, FMT[fmt], _p(out),
                                   _stream(stream)), "moe_test_dequant")
     return out
+
+
+def moe_dequant_experts(w: QWeightT, experts: torch.Tensor, stream=None,
+                        out: torch.Tensor | None = None) -> torch.Tensor:
+    """Whole experts dequantized to BF16: out [count, N, K] = W[experts]."""
+    _require_cuda(experts)
+    count = int(experts.numel())
+    if out is None:
+        out = torch.empty((count, w.N, w.K), dtype=torch.bfloat16, device=experts.device)
+    qw = qweight_c(w)
+    _check(lib().moe_dequant_experts(ctypes.byref(qw), _p(experts), count, _p(out), _stream(stream)),
+           "moe_dequant_experts")
+    return out
+
+
+def moe_ep_regroup(counts: torch.Tensor, rows: torch.Tensor, direction: int, chunk_size: int = 8,
+                   stream=None, out: torch.Tensor | None = None):
+    """Expert parallelism: received rows [R, D] reordered source-major -> local
+    expert-major (direction 0, returns (rows, local Routing tables)) or back
+    (direction 1, returns rows). counts: device int32 [W, E_loc]."""
+    _require_cuda(counts, rows)
+    W, E_loc = counts.shape
+    R, D = rows.shape
+    if out is None:
+        out = torch.empty_like(rows)
+    dev = rows.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    if direction == 0:
+        t = dict(expert_offsets=torch.empty(E_loc + 1, **i32), active=torch.empty(E_loc, **i32),
+                 num_active=torch.empty(1, **i32), chunk_offsets=torch.empty(E_loc + 1, **i32),
+                 num_chunks=torch.empty(1, **i32))
+    else:
+        t = dict(expert_offsets=None, active=None, num_active=None, chunk_offsets=None, num_chunks=None)
+    _check(lib().moe_ep_regroup(_p(counts), W, E_loc, R, _p(rows), _p(out), D, direction, chunk_size,
+                                _p(t["expert_offsets"]), _p(t["active"]), _p(t["num_active"]),
+                                _p(t["chunk_offsets"]), _p(t["num_chunks"]), _stream(stream)),
+           "moe_ep_regroup")
+    if direction == 1:
+        return out
+    groups = Routing(topk_idx=None, gates=None, perm_token=None, inv_perm=None, x_perm=out,
+                     E=E_loc, k=1, **t)
+    return out, groups
 
 
 def moe_test_set_wait_budget(cycles: int):
