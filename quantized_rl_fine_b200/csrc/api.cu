@@ -277,7 +277,7 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   // MOEQ_PIPES=0 turns them off (tuning only).
   pl.pipes = true;
   if (const char* env = getenv("MOEQ_PIPES")) pl.pipes = (atoi(env) != 0);
-  pl.pipes = pl.pipes && pl.lanes == 2 && pl.n_issuers == 2 && !pl.pair;
+  pl.pipes = pl.pipes && pl.n_issuers == 2 && !pl.pair;
   const int stages = pl.stages;
   pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
   const int64_t bound = static_cast<int64_t>(pl.pair ? pl.n_ftiles / 2 : pl.n_ftiles) *

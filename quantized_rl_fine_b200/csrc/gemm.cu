@@ -255,14 +255,15 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int t_first = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int t_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
-  // Tile pipelines (two lanes, two issuers, two producers): the
-  // CTA's i-th tile belongs to pipeline i % 2 as a whole (its producer,
-  // dequant lane and issuer, which accumulates all of its fills in one
-  // accumulator), so one tile's epilogue overlaps the other pipeline's tile.
-  // Otherwise every member takes every other fill of every tile.
-  // (Only with exactly two lanes and two issuers: the planner asks for it
-  // only then, and any other layout would leave a member without tiles.)
-  const bool pipes = !PAIR && LANES == 2 && p.n_issuers == 2 && p.pipes != 0;
+  // Tile pipelines (two issuers, two producers): the CTA's i-th tile belongs
+  // to pipeline i % 2 as a whole: its producer and its issuer, which
+  // accumulates all of the tile's fills in one accumulator, in fill order, so
+  // a token's sum never depends on how the rest of the batch is tiled. With
+  // two lanes, lane i % 2 dequantizes every fill of the tile; with four,
+  // lanes i % 2 and i % 2 + 2 take the pipeline's fills in turn. One tile's
+  // epilogue overlaps the other pipeline's tile. Otherwise (one issuer, or
+  // MOEQ_PIPES=0) every member takes every other fill of every tile.
+  const bool pipes = !PAIR && p.n_issuers == 2 && p.pipes != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -402,14 +403,14 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       }
     }
     // ------------------------------------------------------------ MMA issuers
-    // One thread issuing tcgen05.mma sustains only about one instruction per
-    // ~100 cycles whatever N is, so the reduction of a tile is split among NI
-    // issuing warps: issuer j takes the fills f with f % NI == j into its own
-    // partial accumulator; the epilogue adds the partials in issuer order.
-    // In a pair only the even CTA issues; its MMAs read the A stages and
-    // token rows of both CTAs and write both accumulators, and its commits
-    // arrive on the barriers of both.
-    if (lane == 0 && rank == 0) {
+    // Two issuing warps: with tile pipelines each accumulates whole tiles;
+    // otherwise issuer j takes the fills f with f % NI == j into its own
+    // partial accumulator and the epilogue adds the partials in issuer order.
+    // The whole warp runs the loop and waits; one elected lane issues the
+    // MMAs and commits. In a pair only the even CTA issues; its MMAs read the
+    // A stages and token rows of both CTAs and write both accumulators, and
+    // its commits arrive on the barriers of both.
+    if (rank == 0) {
       const int j = warp - kIssuerWarp0;
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(j * p.acc_cols);
       int st = j, sa = j;                     // stages of the next own fill (f = j, j + NI, ...)
@@ -423,10 +424,13 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       auto mma_ts = [](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t accum) {
         if constexpr (PAIR) mma_bf16_ts_pair(d, a, b, id, accum); else mma_bf16_ts(d, a, b, id, accum);
       };
-      // Barriers the other CTA of a pair arrives on are waited with cluster scope.
+      // Barriers the other CTA of a pair arrives on are waited with cluster
+      // scope. Every lane waits; lane 0's result decides for the warp.
       auto wait_x = [&](uint32_t bar, uint32_t parity) {
-        if constexpr (PAIR) return mbar_wait_cluster(bar, parity, abort_flag);
-        else return mbar_wait(bar, parity, abort_flag);
+        bool r;
+        if constexpr (PAIR) r = mbar_wait_cluster(bar, parity, abort_flag);
+        else r = mbar_wait(bar, parity, abort_flag);
+        return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
       };
       int li = 0;                             // this CTA's tile count
       for (int t = t_first; t < total && ok; t += t_step, ++li) {
@@ -448,40 +452,46 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             if (!wait_x(full_a(sa), pha)) { ok = false; break; }
             tc_fence_after();
             const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
-            if constexpr (kTmemA) {
-              // A stage st: 128 lanes x 64 columns (two BF16 per column): K=16 = 8 columns.
-              const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * 64);
-              const uint64_t b1 = b0 + (b_chunk >> 4);
-              mma_ts(d_tmem, a0, b0, idesc, acc);
-              mma_ts(d_tmem, a0 + 8, b0 + 2, idesc, 1u);
-              mma_ts(d_tmem, a0 + 16, b0 + 4, idesc, 1u);
-              mma_ts(d_tmem, a0 + 24, b0 + 6, idesc, 1u);
-              mma_ts(d_tmem, a0 + 32, b1, idesc, 1u);
-              mma_ts(d_tmem, a0 + 40, b1 + 2, idesc, 1u);
-              mma_ts(d_tmem, a0 + 48, b1 + 4, idesc, 1u);
-              mma_ts(d_tmem, a0 + 56, b1 + 6, idesc, 1u);
-            } else {
-              const uint64_t a0 = smem_desc_sw128(A_at(st), 8192, 1024);
-              mma_bf16_ss(d_tmem, a0, b0, idesc, acc);
-              mma_bf16_ss(d_tmem, a0 + 128, b0 + 2, idesc, 1u);
-              mma_bf16_ss(d_tmem, a0 + 256, b0 + 4, idesc, 1u);
-              mma_bf16_ss(d_tmem, a0 + 384, b0 + 6, idesc, 1u);
+            if (elect_one()) {
+              if constexpr (kTmemA) {
+                // A stage st: 128 lanes x 64 columns (two BF16 per column): K=16 = 8 columns.
+                const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * 64);
+                const uint64_t b1 = b0 + (b_chunk >> 4);
+                mma_ts(d_tmem, a0, b0, idesc, acc);
+                mma_ts(d_tmem, a0 + 8, b0 + 2, idesc, 1u);
+                mma_ts(d_tmem, a0 + 16, b0 + 4, idesc, 1u);
+                mma_ts(d_tmem, a0 + 24, b0 + 6, idesc, 1u);
+                mma_ts(d_tmem, a0 + 32, b1, idesc, 1u);
+                mma_ts(d_tmem, a0 + 40, b1 + 2, idesc, 1u);
+                mma_ts(d_tmem, a0 + 48, b1 + 4, idesc, 1u);
+                mma_ts(d_tmem, a0 + 56, b1 + 6, idesc, 1u);
+              } else {
+                const uint64_t a0 = smem_desc_sw128(A_at(st), 8192, 1024);
+                mma_bf16_ss(d_tmem, a0, b0, idesc, acc);
+                mma_bf16_ss(d_tmem, a0 + 128, b0 + 2, idesc, 1u);
+                mma_bf16_ss(d_tmem, a0 + 256, b0 + 4, idesc, 1u);
+                mma_bf16_ss(d_tmem, a0 + 384, b0 + 6, idesc, 1u);
+              }
+              commit(empty(st));
+              if constexpr (kTmemA) commit(a_free(sa));
             }
+            __syncwarp();
             acc = 1u;
-            commit(empty(st));
-            if constexpr (kTmemA) commit(a_free(sa));
           }
           st += NI;
           if (st >= S) st -= S;
           sa += NI;
           if (sa >= SA) { sa -= SA; pha ^= 1u; }
         }
-        if (ok) commit(acc_full(q_acc));      // arrives even when this issuer had no fill
+        if (ok && elect_one()) commit(acc_full(q_acc));   // arrives even when this issuer had no fill
+        __syncwarp();
         ++it;                                 // tiles this issuer has handed over
       }
       // All MMAs of this CTA (of the pair) done before tensor memory is released.
-      commit(drain_bar);
-      mbar_drain(drain_bar, 0);
+      if (elect_one()) commit(drain_bar);
+      __syncwarp();
+      if (lane == 0) mbar_drain(drain_bar, 0);
+      __syncwarp();
     }
   } else if (warp >= kDqWarp0 && warp < kDqWarp0 + kLanes * kDqWarpsPerLane) {
     // ------------------------------------------------------------ dequantizers
@@ -502,6 +512,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     // owns fills grp, grp + kLanes, ... and steps its stage and parity
     // incrementally.
     int r0 = 0;                             // (first fill of the tile) % kLanes
+    // With tile pipelines: lanes grp % 2 + 2 h (h < kLanes / 2) serve pipeline
+    // grp % 2, taking its fills n (counted across the pipeline's tiles) with
+    // n % (kLanes / 2) == h; rp = (fills of the pipeline so far) % (kLanes / 2).
+    constexpr int kPipeLanes = kLanes / 2;
+    const int pipe_of = grp & 1, pipe_h = grp >> 1;
+    int rp = 0;
     int st = grp, sa = grp;                 // fill ring and A ring positions of the next own fill
     uint32_t ph = 0, pha = 0;
     bool ok = true;
@@ -510,9 +526,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       int kb_first = (grp - r0 + kLanes) % kLanes, kb_step = kLanes;
       r0 = (r0 + nkb) % kLanes;
       if (pipes) {
-        if ((li & 1) != grp) continue;
-        kb_first = 0;
-        kb_step = 1;
+        if ((li & 1) != pipe_of) continue;
+        kb_first = (pipe_h - rp + kPipeLanes) % kPipeLanes;
+        kb_step = kPipeLanes;
+        rp = (rp + nkb) % kPipeLanes;
       }
       for (int kb = kb_first; kb < nkb; kb += kb_step) {
         const int cur = st, cur_a = sa;
