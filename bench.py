@@ -396,11 +396,12 @@ def _step_fn(cfg, chunk):
 
 
 def _launches_per_step(cfg):
-    # routing: top-k and the tail (which also copies the rows) for launches of
-    # at most 1024 tokens whose token-by-expert bit matrix fits 8192 words;
-    # else top-k, scan, scatter and the row copy
+    # routing: top-k and the single-pass tail for launches of at most 1024
+    # tokens whose token-by-expert bit matrix fits 8192 words; else top-k,
+    # scan and scatter. The permuted rows are not copied: the gate/up GEMM
+    # (or the adapter) gathers them.
     words = (cfg.T + 31) // 32
-    route = 2 if words <= 32 and words * cfg.E <= 8192 else 4
+    route = 2 if words <= 32 and words * cfg.E <= 8192 else 3
     if not cfg.swiglu:
         return route + 1
     n = route + 2 + 1                           # gate/up, down, combine
@@ -511,25 +512,29 @@ def run_ours(args, cfg):
         r = st["routing"]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
+            # the layer's call: row p of the input is x[perm_token[p]]
             if not cfg.swiglu:
-                moeq.moe_grouped_qgemm_fwd(r.x_perm, wl["w_up"], r, moeq.EPI_NONE)
+                moeq.moe_grouped_qgemm_fwd(wl["x"], wl["w_up"], r, moeq.EPI_NONE,
+                                           a_rows=r.perm_token)
             else:
-                moeq.moe_grouped_qgemm_fwd(r.x_perm, wl["w_gu"], r, moeq.EPI_SWIGLU,
-                                           adapter=wl.get("adapter"), save_gu=cfg.train)
+                moeq.moe_grouped_qgemm_fwd(wl["x"], wl["w_gu"], r, moeq.EPI_SWIGLU,
+                                           adapter=wl.get("adapter"), save_gu=cfg.train,
+                                           a_rows=r.perm_token)
         gemm_graphs.append(g)
     for i in range(max(3, args.warmup)):
         gemm_graphs[i % ROTATE].replay()
     torch.cuda.synchronize()
     ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    # At least 200 launches and 200 ms, whatever --steps is, so the kernel's
-    # time does not depend on how long the step timing ran.
+    # About 200 ms of back-to-back launches (at least 20), whatever --steps
+    # is, so the kernel's time does not depend on how long the step timing
+    # ran and every workload's kernel is timed over the same span.
     ka.record(stream)
     for i in range(10):
         gemm_graphs[i % ROTATE].replay()
     kb.record(stream)
     torch.cuda.synchronize()
     est_ms = ka.elapsed_time(kb) / 10
-    n_k = max(200, int(200.0 / max(est_ms, 1e-3)) + 1)
+    n_k = max(20, int(200.0 / max(est_ms, 1e-3)) + 1)
     ka.record(stream)
     for i in range(n_k):
         gemm_graphs[i % ROTATE].replay()
@@ -694,12 +699,14 @@ def run_prior_art(args, cfg):
         h = torch.empty((M, cfg.f), dtype=torch.bfloat16, device=dev)
         y = torch.empty((M, cfg.d if cfg.swiglu else cfg.f), dtype=torch.bfloat16, device=dev)
 
-        def fused():
+        def fused():   # the layer's calls: rows gathered from x in the kernel
             if cfg.swiglu:
-                moeq.moe_grouped_qgemm_fwd(r.x_perm, w_first, r, moeq.EPI_SWIGLU, out=h)
+                moeq.moe_grouped_qgemm_fwd(wl["x"], w_first, r, moeq.EPI_SWIGLU, out=h,
+                                           a_rows=r.perm_token)
                 moeq.moe_grouped_qgemm_fwd(h, wl["w_d"], r, moeq.EPI_NONE, out=y)
             else:
-                moeq.moe_grouped_qgemm_fwd(r.x_perm, w_first, r, moeq.EPI_NONE, out=y)
+                moeq.moe_grouped_qgemm_fwd(wl["x"], w_first, r, moeq.EPI_NONE, out=y,
+                                           a_rows=r.perm_token)
         got = {}
 
         def prior():

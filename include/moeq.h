@@ -198,7 +198,13 @@ moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t
  * block-diagonal matrix of adapter[e][b] (32 x 32 blocks, row-vector
  * convention, x'[32b+j] = sum_i x[32b+i] R[e][b][i][j]).
  *
- *  a        [M][K] bf16 permuted rows (x_perm), grouped by expert offsets.
+ *  a        [M][K] bf16 permuted rows (x_perm), grouped by expert offsets;
+ *           or, with a_rows, the token rows [T][K] themselves.
+ *  a_rows   NULL, or device int32 [M]: row p of the GEMM input is
+ *           a[a_rows[p]] (perm_token from moe_route_permute). The kernels
+ *           then gather the rows as they go, and the permuted rows never
+ *           need to be written to memory (moe_route_permute may be called
+ *           with x = NULL). Each index must be a valid row of a.
  *  w        frozen weights, W[e] is [N][K].
  *  g        groups from moe_route_permute; g->E == w->E, off[E] == M.
  *  adapter  NULL or [E][K/32][32][32] bf16.
@@ -209,10 +215,10 @@ moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t
  *  ws       scratch: M*K bf16 for a' with an adapter; none without one.
  * Experts with no rows cost nothing: their weight bytes are never read.
  */
-moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
-                                 const moe_groups* g, const void* adapter, int32_t epi,
-                                 void* out, void* saved_gu, void* ws, size_t* ws_bytes,
-                                 void* stream);
+moe_status moe_grouped_qgemm_fwd(const void* a, const int32_t* a_rows, int64_t M,
+                                 const moe_qweight* w, const moe_groups* g, const void* adapter,
+                                 int32_t epi, void* out, void* saved_gu, void* ws,
+                                 size_t* ws_bytes, void* stream);
 
 /*
  * moe_grouped_qgemm_bwd_dx -- activation-gradient grouped GEMM; the frozen
@@ -231,12 +237,15 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
  *             s = sigmoid(g): din [M][2K] = bf16([dh*u*s*(1+g*(1-s)) |
  *             dh*g*s]). adapter must be NULL.
  *  adapter, a, d_adapter: NULL, or all three given (a = the forward's a).
+ *  a_rows   NULL, or device int32 [M] as in moe_grouped_qgemm_fwd: row p of
+ *           the adapter's input is a[a_rows[p]] (only with an adapter).
  *  ws       scratch: M*K bf16 for dx' with an adapter; none without one.
  */
 moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweight* w,
                                     const moe_groups* g, int32_t epi, const void* saved_gu,
-                                    const void* adapter, const void* a, void* din,
-                                    float* d_adapter, void* ws, size_t* ws_bytes, void* stream);
+                                    const void* adapter, const void* a, const int32_t* a_rows,
+                                    void* din, float* d_adapter, void* ws, size_t* ws_bytes,
+                                    void* stream);
 
 /*
  * moe_unpermute_combine -- the two row moves around the grouped GEMMs.
@@ -327,7 +336,7 @@ moe_status moe_test_dequant(const void* packed, const void* scales, int64_t R, i
                             int32_t fmt, void* out, void* stream);
 moe_status moe_test_set_wait_budget(int64_t cycles);
 
-#define MOEQ_ABI_VERSION 1
+#define MOEQ_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

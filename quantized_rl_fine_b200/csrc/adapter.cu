@@ -98,10 +98,13 @@ __device__ __forceinline__ void load_r_frags(const __nv_bfloat16* __restrict__ R
 // expert's R block, as B fragments, stays in registers while the rows'
 // expert does not change; a group whose rows span several experts runs the
 // MMAs once per expert and keeps each row's result from its own expert.
-// TRANS = 0: out = x . R_e; 1: out = x . R_e^T.
+// TRANS = 0: out = x . R_e; 1: out = x . R_e^T. With rows (not NULL) the
+// task's row p reads x[rows[p]] (the permuted rows are gathered from the token
+// rows here, so they are never written out).
 template <int TRANS>
 __global__ void __launch_bounds__(256)
-adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ R,
+adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ rows,
+                     const __nv_bfloat16* __restrict__ R,
                      const int32_t* __restrict__ offsets, int E, int M, int K,
                      __nv_bfloat16* __restrict__ out) {
   grid_dependency_wait();
@@ -123,7 +126,8 @@ adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
     for (int h = 0; h < 8; ++h) {
       const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
       const int r = span0 + row;
-      v[h] = (r < M) ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(r) * K + 32 * b + 8 * ch))
+      const int64_t src = (r < M) ? (rows ? __ldg(rows + r) : r) : 0;
+      v[h] = (r < M) ? __ldg(reinterpret_cast<const uint4*>(x + src * K + 32 * b + 8 * ch))
                      : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
@@ -213,7 +217,8 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
 // so dx' is read from HBM once for both. dx is staged where the x rows were
 // and written with 16-byte stores.
 __global__ void __launch_bounds__(256)
-adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ dxp,
+adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ rows,
+                   const __nv_bfloat16* __restrict__ dxp,
                    const __nv_bfloat16* __restrict__ R, const int32_t* __restrict__ offsets,
                    int K, __nv_bfloat16* __restrict__ dx, float* __restrict__ dR) {
   grid_dependency_wait();
@@ -246,8 +251,10 @@ adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
     for (int h = 0; h < 4; ++h) {
       const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
       const bool ok = c0 + row < p1;
-      const int64_t gi = static_cast<int64_t>(ok ? c0 + row : p0) * K + 32 * b + 8 * ch;
-      vx[h] = ok ? __ldg(reinterpret_cast<const uint4*>(x + gi)) : make_uint4(0, 0, 0, 0);
+      const int pr = ok ? c0 + row : p0;
+      const int64_t gi = static_cast<int64_t>(pr) * K + 32 * b + 8 * ch;
+      const int64_t xi = (rows ? static_cast<int64_t>(__ldg(rows + pr)) : pr) * K + 32 * b + 8 * ch;
+      vx[h] = ok ? __ldg(reinterpret_cast<const uint4*>(x + xi)) : make_uint4(0, 0, 0, 0);
       vg[h] = ok ? __ldg(reinterpret_cast<const uint4*>(dxp + gi)) : make_uint4(0, 0, 0, 0);
     }
     __syncwarp();                        // the previous step's stores from xs are done
@@ -331,25 +338,26 @@ adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __r
 
 }  // namespace
 
-cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* offsets, int E,
-                                 int M, int K, void* out, cudaStream_t s) {
+cudaError_t launch_adapter_apply(const void* x, const int32_t* rows, const void* R,
+                                 const int32_t* offsets, int E, int M, int K, void* out,
+                                 cudaStream_t s) {
   if (M == 0) return cudaSuccess;
   const int nb = K / 32;
   const int64_t spans = (static_cast<int64_t>(M) + 16 * kApplyGroups - 1) / (16 * kApplyGroups);
   const int64_t ctas = (spans * nb + 7) / 8;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   return launch_pdl(adapter_apply_kernel<0>, dim3(static_cast<unsigned>(ctas)), dim3(256), 0, s,
-                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(R),
+                    static_cast<const __nv_bfloat16*>(x), rows, static_cast<const __nv_bfloat16*>(R),
                     offsets, E, M, K, static_cast<__nv_bfloat16*>(out));
 }
 
-cudaError_t launch_adapter_bwd(const void* x, const void* dxp, const void* R,
+cudaError_t launch_adapter_bwd(const void* x, const int32_t* rows, const void* dxp, const void* R,
                                const int32_t* offsets, int E, int K, void* dx, float* dR,
                                cudaStream_t s) {
   const int nb = K / 32;
   dim3 grid(E, (nb + kGradWarps - 1) / kGradWarps);
   return launch_pdl(adapter_bwd_kernel, grid, dim3(256), 0, s,
-                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(dxp),
+                    static_cast<const __nv_bfloat16*>(x), rows, static_cast<const __nv_bfloat16*>(dxp),
                     static_cast<const __nv_bfloat16*>(R), offsets, K,
                     static_cast<__nv_bfloat16*>(dx), dR);
 }

@@ -170,9 +170,10 @@ moe_status check_groups(const moe_groups* g, int E) {
 }
 
 struct GemmPlan {
-  int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers, lanes;
-  bool pair;   // forward on CTA pairs (M = 256 MMAs)
-  bool pipes;  // two tile pipelines per CTA
+  int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers, lanes, dq_warps;
+  bool pair;    // forward on CTA pairs (M = 256 MMAs)
+  bool pipes;   // two tile pipelines per CTA
+  bool halves;  // forward: A stages handed over in 64-wide halves
   uint32_t stage_bytes;
   size_t smem;
 };
@@ -220,6 +221,12 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
     const int v = atoi(env);
     if (v == 2 || v == 4) pl.lanes = v;
   }
+  // Dequant warps: sixteen; eight (one per lane quarter and lane, a whole
+  // 128-wide fill per thread) with two lanes when MOEQ_DQW=8 (tuning).
+  pl.dq_warps = 16;
+  if (const char* env = getenv("MOEQ_DQW")) {
+    if (atoi(env) == 8 && pl.lanes == 2 && !pl.pair) pl.dq_warps = 8;
+  }
   const int L = pl.lanes;
   // Every ring has a multiple of L stages, and of n_issuers where the issuers
   // wait on it (the A ring), so that each stage has one waiter per role.
@@ -236,9 +243,17 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   };
   if (mode == kModeFwd) {
     // A stage of a 128-wide fill: 64 tensor-memory columns. The most issuers
-    // that still leave four A stages (one issuer always does, as BN <= 96).
+    // that still leave four A stages; with two issuers and wide accumulators
+    // (more than 128 columns each) two A stages, handed over in halves, so
+    // that a pipeline's next fill is dequantized while its previous fill's
+    // second half is multiplied. MOEQ_HALVES=0/1 overrides (tuning).
+    int halves_env = -1;
+    if (const char* env = getenv("MOEQ_HALVES")) halves_env = atoi(env) != 0 ? 1 : 0;
+    bool pipes_allowed = true;
+    if (const char* env = getenv("MOEQ_PIPES")) pipes_allowed = (atoi(env) != 0);
     pl.n_issuers = 1;
     pl.a_stages = 4;
+    pl.halves = false;
     for (int ni = ni_max; ni >= 1; --ni) {
       const int step = ring_step(ni);
       const int room = (512 - ni * pl.acc_cols) / 64;
@@ -246,6 +261,13 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
       if (sa >= 4) {
         pl.n_issuers = ni;
         pl.a_stages = sa;
+        pl.halves = halves_env == 1;
+        break;
+      }
+      if (ni == 2 && sa >= 2 && halves_env != 0 && pipes_allowed) {
+        pl.n_issuers = ni;
+        pl.a_stages = sa;
+        pl.halves = true;
         break;
       }
     }
@@ -259,6 +281,7 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
     while (stages > L && !fits(stages, pl.a_stages)) stages -= L;
     pl.stages = stages;
   } else {
+    pl.halves = false;
     int stages = 16;
     while (stages > L && !fits(stages, stages)) stages -= L;
     pl.stages = stages;
@@ -277,7 +300,7 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   // MOEQ_PIPES=0 turns them off (tuning only).
   pl.pipes = true;
   if (const char* env = getenv("MOEQ_PIPES")) pl.pipes = (atoi(env) != 0);
-  pl.pipes = pl.pipes && pl.n_issuers == 2 && !pl.pair;
+  pl.pipes = pl.pipes && pl.n_issuers == 2;
   const int stages = pl.stages;
   pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
   const int64_t bound = static_cast<int64_t>(pl.pair ? pl.n_ftiles / 2 : pl.n_ftiles) *
@@ -311,7 +334,7 @@ moe_status check_workspace(void* ws, size_t* ws_bytes, size_t need) {
 // Runs one grouped GEMM launch over the rows of `bmat` (a, a' or dout).
 moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qweight* w,
                     const moe_groups* g, void* out, int64_t ldo, void* saved, const GemmPlan& pl,
-                    cudaStream_t s) {
+                    cudaStream_t s, const int32_t* b_rows = nullptr) {
   const int F = (mode == kModeFwd) ? (epi == MOE_EPI_SWIGLU ? w->N / 2 : w->N) : w->K;
   const int R = (mode == kModeFwd) ? w->K : w->N;
   CUtensorMap tb, tw, ts;
@@ -383,10 +406,17 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   p.a_stages = pl.a_stages;
   p.stage_bytes = pl.stage_bytes;
   p.pipes = pl.pipes ? 1 : 0;
+  p.a_halves = pl.halves ? 1 : 0;
+  // Gathered rows: the token-row tensor map above is encoded (over the same
+  // base) but not read; the producers copy row b_rows[p] of bmat instead.
+  p.b_rows = b_rows;
+  p.b_src = static_cast<const __nv_bfloat16*>(bmat);
+  if (b_rows && pl.stages < 4) return MOE_ERR_UNSUPPORTED;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.ldo = ldo;
   p.saved = static_cast<__nv_bfloat16*>(saved);
-  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, pl.lanes, pl.pair, tb, tw, ts, p, pl.grid, pl.smem, s));
+  return cuda_status(launch_grouped_qgemm(mode, w->fmt, epi, pl.lanes, pl.dq_warps, pl.pair, tb, tw,
+                                          ts, p, pl.grid, pl.smem, s));
 }
 
 }  // namespace
@@ -525,9 +555,10 @@ moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t
                                   static_cast<cudaStream_t>(stream)));
 }
 
-moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
-                                 const moe_groups* g, const void* adapter, int32_t epi, void* out,
-                                 void* saved_gu, void* ws, size_t* ws_bytes, void* stream) {
+moe_status moe_grouped_qgemm_fwd(const void* a, const int32_t* a_rows, int64_t M,
+                                 const moe_qweight* w, const moe_groups* g, const void* adapter,
+                                 int32_t epi, void* out, void* saved_gu, void* ws,
+                                 size_t* ws_bytes, void* stream) {
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -541,32 +572,34 @@ moe_status moe_grouped_qgemm_fwd(const void* a, int64_t M, const moe_qweight* w,
   if ((st = check_groups(g, w->E)) != MOE_OK) return st;
   if (!a || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(out) || (saved_gu && !aligned16(saved_gu)) ||
-      (adapter && !aligned16(adapter)))
+      (adapter && !aligned16(adapter)) || (a_rows && !aligned16(a_rows)))
     return MOE_ERR_MISALIGNED;
   if (saved_gu && epi != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const void* bmat = a;
   if (adapter) {
+    // The adapter kernel gathers the rows (a_rows) and writes a' in expert
+    // order; the GEMM then reads a' through its tensor map.
     void* xa = ws;
-    cudaError_t e = launch_adapter_apply(a, adapter, g->expert_offsets, w->E, static_cast<int>(M),
-                                         w->K, xa, s);
+    cudaError_t e = launch_adapter_apply(a, a_rows, adapter, g->expert_offsets, w->E,
+                                         static_cast<int>(M), w->K, xa, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    bmat = xa;
+    return run_gemm(kModeFwd, epi, xa, M, w, g, out, F, saved_gu, pl, s);
   }
-  return run_gemm(kModeFwd, epi, bmat, M, w, g, out, F, saved_gu, pl, s);
+  return run_gemm(kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s, a_rows);
 }
 
 moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweight* w,
                                     const moe_groups* g, int32_t epi, const void* saved_gu,
-                                    const void* adapter, const void* a, void* din,
-                                    float* d_adapter, void* ws, size_t* ws_bytes, void* stream) {
+                                    const void* adapter, const void* a, const int32_t* a_rows,
+                                    void* din, float* d_adapter, void* ws, size_t* ws_bytes,
+                                    void* stream) {
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
   if (epi != MOE_EPI_NONE && epi != MOE_EPI_SWIGLU_BWD) return MOE_ERR_INVALID_ARG;
   const bool with_adapter = adapter != nullptr;
   if (with_adapter && (epi != MOE_EPI_NONE || !a || !d_adapter)) return MOE_ERR_INVALID_ARG;
-  if (!with_adapter && (a || d_adapter)) return MOE_ERR_INVALID_ARG;
+  if (!with_adapter && (a || a_rows || d_adapter)) return MOE_ERR_INVALID_ARG;
   if (epi == MOE_EPI_SWIGLU_BWD && !saved_gu) return MOE_ERR_INVALID_ARG;
   const GemmPlan pl = plan_gemm(kModeBwd, M, w, w->K, 128, w->fmt);
   const size_t need = with_adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
@@ -576,7 +609,7 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
   if (!dout || !din) return MOE_ERR_INVALID_ARG;
   if (!aligned16(dout) || !aligned16(din) || (saved_gu && !aligned16(saved_gu)) ||
       (adapter && !aligned16(adapter)) || (a && !aligned16(a)) ||
-      (d_adapter && !aligned16(d_adapter)))
+      (a_rows && !aligned16(a_rows)) || (d_adapter && !aligned16(d_adapter)))
     return MOE_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (epi == MOE_EPI_SWIGLU_BWD) {
@@ -589,8 +622,8 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
   void* dxa = ws;
   st = run_gemm(kModeBwd, epi, dout, M, w, g, dxa, w->K, nullptr, pl, s);
   if (st != MOE_OK) return st;
-  return cuda_status(launch_adapter_bwd(a, dxa, adapter, g->expert_offsets, w->E, w->K, din,
-                                        d_adapter, s));
+  return cuda_status(launch_adapter_bwd(a, a_rows, dxa, adapter, g->expert_offsets, w->E, w->K,
+                                        din, d_adapter, s));
 }
 
 moe_status moe_unpermute_combine(const void* rows, const int32_t* inv_perm, const float* gates,

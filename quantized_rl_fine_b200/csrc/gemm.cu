@@ -47,9 +47,10 @@ namespace moeq {
 
 namespace {
 
-constexpr int kThreads = kGemmThreads;
-// 24 warps: six on each of the four SM sub-partitions, so 80 registers a thread.
-static_assert(kThreads <= 1024 && ((kThreads / 32 + 3) / 4) * 32 * 80 <= 16384, "roles must fit 80 registers a thread");
+// 24 warps (16 dequant warps): six on each of the four SM sub-partitions, so
+// 80 registers a thread; 16 warps (8 dequant warps): 128 registers a thread.
+static_assert(gemm_threads(16) <= 1024 && ((gemm_threads(16) / 32 + 3) / 4) * 32 * 80 <= 16384,
+              "roles must fit 80 registers a thread");
 constexpr int kTileF = 128;            // output features per tile (MMA M)
 constexpr uint32_t kABytes = kTileF * 64 * 2;   // 16 KiB dequantized A tile (backward fill)
 
@@ -184,12 +185,14 @@ __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* 
 __device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int MODE, int FMT, int EPI, int LANES, int PAIR>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MODE, int FMT, int EPI, int LANES, int PAIR, int DQW>
+__global__ void __launch_bounds__(gemm_threads(DQW), 1)
 grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
                      const __grid_constant__ CUtensorMap tm_wq,
                      const __grid_constant__ CUtensorMap tm_sc, const GemmArgs p) {
   constexpr int kLanes = LANES;
+  constexpr int kDqWarps = DQW;
+  constexpr int kEpiWarp0 = kDqWarp0 + kDqWarps;
   constexpr int kDqWarpsPerLane = kDqWarps / LANES;   // 4 or 8
   constexpr int kParts = kDqWarpsPerLane / 4;         // warps per lane quarter
   static_assert(LANES % kProdWarps == 0 && LANES % kMaxIssuers == 0, "lanes own their stages");
@@ -231,17 +234,24 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   // kernels the A stages live in tensor memory and may be fewer than the
   // fills; in the backward kernels the A tile is part of the fill (SA = S).
   const int SA = p.a_stages;
+  // Forward with A halves: each A stage (64 tensor-memory columns, a 128-wide
+  // fill) is handed over in two 64-wide halves, each with its own pair of
+  // barriers, so the MMAs of a fill's first half start as soon as it is
+  // dequantized and the next fill's first half may be written while the
+  // second half's MMAs run. A-barrier j of stage sa is 2 sa + half.
+  const bool halves = kTmemA && p.a_halves != 0;
+  const int SAB = 2 * SA;                          // A-barrier slots reserved (two per stage)
   const uint32_t bars = base + S * stage_bytes;
   auto full_tma = [&](int s) { return bars + 8u * s; };
   auto empty = [&](int s) { return bars + 8u * (S + s); };
   auto full_a = [&](int s) { return bars + 8u * (2 * S + s); };
-  auto a_free = [&](int s) { return bars + 8u * (2 * S + SA + s); };
+  auto a_free = [&](int s) { return bars + 8u * (2 * S + SAB + s); };
   // Accumulator handoff: one pair of barriers per pipeline (two with tile
   // pipelines, else only the first is used).
-  auto acc_full = [&](int q) { return bars + 8u * (2 * S + 2 * SA + q); };
-  auto acc_empty = [&](int q) { return bars + 8u * (2 * S + 2 * SA + 2 + q); };
-  const uint32_t drain_bar = bars + 8u * (2 * S + 2 * SA + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (2 * S + 2 * SA + 5));
+  auto acc_full = [&](int q) { return bars + 8u * (2 * S + 2 * SAB + q); };
+  auto acc_empty = [&](int q) { return bars + 8u * (2 * S + 2 * SAB + 2 + q); };
+  const uint32_t drain_bar = bars + 8u * (2 * S + 2 * SAB + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + S * stage_bytes + 8u * (2 * S + 2 * SAB + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* warp_tot = reinterpret_cast<int32_t*>(tmem_slot + 4);          // [32]
   int32_t* tile_start = warp_tot + 32;                                      // [E + 1]
@@ -263,23 +273,30 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   // lanes i % 2 and i % 2 + 2 take the pipeline's fills in turn. One tile's
   // epilogue overlaps the other pipeline's tile. Otherwise (one issuer, or
   // MOEQ_PIPES=0) every member takes every other fill of every tile.
-  const bool pipes = !PAIR && p.n_issuers == 2 && p.pipes != 0;
+  const bool pipes = p.n_issuers == 2 && p.pipes != 0;
+  // Forward, token rows gathered through an index instead of a tensor map.
+  const bool gather = MODE == kModeFwd && p.b_rows != nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full_tma(s), 1);
+      // Gathered token rows: the producer's arrival with the weights' byte
+      // count, and its arrival once the stage's row copies have landed.
+      mbar_init(full_tma(s), gather ? 2 : 1);
       mbar_init(empty(s), 1);
     }
-    for (int s = 0; s < SA; ++s) {
-      // A pair's odd CTA relays its dequant arrivals to the even CTA with one
-      // remote arrival per stage (its own warps arrive locally).
-      mbar_init(full_a(s), (PAIR && rank == 0) ? kDqWarpsPerLane + 1 : kDqWarpsPerLane);
+    // Arrivals on an A barrier: every dequant warp of the lane, or, with
+    // halves and two warps per lane quarter, the four warps of that half. A
+    // pair's odd CTA relays its dequant arrivals to the even CTA with one
+    // remote arrival per barrier (its own warps arrive locally).
+    const int dq_arrivals = (halves && kParts == 2) ? kDqWarpsPerLane / 2 : kDqWarpsPerLane;
+    for (int s = 0; s < (halves ? SAB : SA); ++s) {
+      mbar_init(full_a(s), (PAIR && rank == 0) ? dq_arrivals + 1 : dq_arrivals);
       mbar_init(a_free(s), 1);
     }
     mbar_init(acc_full(0), pipes ? 1 : p.n_issuers);
     mbar_init(acc_full(1), 1);
     mbar_init(acc_empty(0), PAIR ? 8 : 4);
-    mbar_init(acc_empty(1), 4);
+    mbar_init(acc_empty(1), PAIR ? 8 : 4);
     mbar_init(drain_bar, p.n_issuers);
     *abort_flag = 0;
     fence_barrier_init();
@@ -318,7 +335,111 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const int NI = p.n_issuers;
   const uint32_t a_col0 = static_cast<uint32_t>(NI * p.acc_cols);
 
-  if (warp < kProdWarps) {
+  if (warp < kProdWarps && gather) {
+    // ------------------------------------------------------------ gathering producers
+    // The whole warp copies the stage's token rows, 16 bytes a lane, from the
+    // token rows b_src[b_rows[p]] into the 128B-swizzled [2 chunks][rows][64]
+    // layout the tensor map would have written (16-byte unit u of row r at
+    // unit u ^ (r % 8)), zero-filling rows past the tile and a reduction tail
+    // past R; lane 0 issues the weight and scale copies. The row copies run in
+    // the generic proxy and the MMAs read them through the async proxy, so a
+    // stage is handed over only after its copies have completed and the lane
+    // has fenced between the proxies: each fill's copies form one group, and
+    // the previous own fill is signalled once only the newest group is in
+    // flight (the ring has at least four stages, so this never waits on a
+    // fill it has not released).
+    const int pw = warp;
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint32_t tx = kWqFill + kScFill;
+    int st = pw;
+    uint32_t ph = 0;
+    int pending = -1;                        // stage of the own fill not yet signalled
+    long long g_next = pw, last_own = -1;    // ring index of the next / last issued own fill
+    int r0 = 0;
+    bool ok = true;
+    int li = 0;
+    constexpr int kTokRegs = 8;              // 32-row blocks of a tile (at most 256 rows)
+    for (int t = t_first; t < total && ok; t += t_step, ++li) {
+      int kb0 = (pw - r0 + kProdWarps) % kProdWarps, kbs = kProdWarps;
+      r0 = (r0 + nkb) % kProdWarps;
+      if (pipes) {
+        if ((li & 1) != pw) continue;
+        kb0 = 0;
+        kbs = 1;
+      }
+      const Tile tl = tile_at(t);
+      const int rows_here = PAIR ? (tl.width >> 1) : tl.width;
+      const int brow = tl.row0 + static_cast<int>(rank) * rows_here;
+      // Lane l holds the token of rows l, l + 32, ... of this CTA's share (-1 past the expert).
+      int tok[kTokRegs];
+#pragma unroll
+      for (int j = 0; j < kTokRegs; ++j) {
+        const int rr = 32 * j + lane;
+        tok[j] = (rr < rows_here && brow + rr < tl.row_end) ? __ldg(p.b_rows + brow + rr) : -1;
+      }
+      for (int kb = kb0; kb < nkb; kb += kbs) {
+        bool w_ok = true;
+        if (lane == 0) w_ok = mbar_wait(empty(st), ph ^ 1u, abort_flag);
+        if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) { ok = false; break; }
+        const uint32_t bar = full_tma(st);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar, tx);
+          if constexpr (EPI == MOE_EPI_SWIGLU) {
+            tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * 64, tl.ft * 64, 2 * tl.e, pol_w);
+            tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * 64, 0, tl.e * (K / 32) + kb * 4, pol_w);
+          } else {
+            tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * 64, tl.e * N + tl.ft * kTileF, 0, pol_w);
+            tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * kTileF, tl.e * (K / 32) + kb * 4, 0, pol_w);
+          }
+        }
+        // Row rl of a 32-row block: lanes 0-15 row 2 mm, lanes 16-31 row 2 mm + 1;
+        // lanes 8-15 (24-31) the second 64-element chunk; unit u = lane % 8.
+        const int c = (lane >> 3) & 1, u = lane & 7;
+        const bool k_ok = kb * kFillK + c * 64 < p.R;
+        const uint32_t bst = B_at(st) + static_cast<uint32_t>(c) * b_chunk;
+#pragma unroll
+        for (int j = 0; j < kTokRegs; ++j) {
+          if (32 * j >= rows_here) break;
+#pragma unroll 4
+          for (int mm = 0; mm < 16; ++mm) {
+            const int rl = 2 * mm + (lane >> 4);
+            const int r = 32 * j + rl;
+            const int tk = __shfl_sync(0xffffffffu, tok[j], rl);
+            const bool valid = k_ok && tk >= 0;
+            const __nv_bfloat16* src =
+                p.b_src + (valid ? static_cast<int64_t>(tk) * p.R + kb * kFillK + c * 64 + u * 8 : 0);
+            if (r < rows_here)
+              cp_async_16(bst + static_cast<uint32_t>(r) * 128u + ((u ^ (r & 7)) << 4), src,
+                          valid ? 16u : 0u);
+          }
+        }
+        cp_async_commit();
+        if (pending >= 0) {
+          cp_async_wait<1>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full_tma(pending));
+        }
+        pending = st;
+        last_own = g_next;
+        g_next += kProdWarps;
+        st += kProdWarps;
+        if (st >= S) { st -= S; ph ^= 1u; }
+      }
+    }
+    // The last own fill (also after an abort: its copies land, then it is
+    // signalled, so no consumer waits on it in vain and no copy outlives the CTA).
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (pending >= 0 && lane == 0) mbar_arrive(full_tma(pending));
+    if (!ok && lane == 0) {
+      // Weight copies that may still be in flight (own fills within the last
+      // S) land before the CTA can exit: each such stage's phase completes.
+      for (long long g = last_own; g >= 0 && g > last_own - S; g -= kProdWarps)
+        mbar_drain(full_tma(static_cast<int>(g % S)), static_cast<uint32_t>((g / S) & 1));
+    }
+  } else if (warp < kProdWarps) {
     // ------------------------------------------------------------ TMA producers
     // Producer pw issues fills f with f % kProdWarps == pw: one thread issues
     // the fill's three bulk tensor copies (token rows, packed weights, group
@@ -389,15 +510,24 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       // for each A stage of this CTA to be complete (its dequant warps
       // arrive locally) and passes that on with a single arrival on the even
       // CTA's barrier of the stage.
-      if (rank == 1 && warp == kIssuerWarp0 && lane == 0) {
-        int sa = 0;
+      // With tile pipelines, issuer warp j's lane relays pipeline j's fills.
+      const int j = warp - kIssuerWarp0;
+      if (rank == 1 && lane == 0 && (pipes || j == 0)) {
+        int sa = pipes ? j : 0;
+        const int sa_step = pipes ? NI : 1;
         uint32_t pha = 0;
         bool ok = true;
-        for (int t = t_first; t < total && ok; t += t_step) {
-          for (int kb = 0; kb < nkb; ++kb) {
-            if (!mbar_wait(full_a(sa), pha, abort_flag)) { ok = false; break; }
-            mbar_arrive_cluster(cluster_addr(full_a(sa), 0));
-            if (++sa == SA) { sa = 0; pha ^= 1u; }
+        int li = 0;
+        for (int t = t_first; t < total && ok; t += t_step, ++li) {
+          if (pipes && (li & 1) != j) continue;
+          for (int kb = 0; kb < nkb && ok; ++kb) {
+            for (int h = 0; h < (halves ? 2 : 1); ++h) {
+              const int jb = halves ? 2 * sa + h : sa;
+              if (!mbar_wait(full_a(jb), pha, abort_flag)) { ok = false; break; }
+              mbar_arrive_cluster(cluster_addr(full_a(jb), 0));
+            }
+            sa += sa_step;
+            if (sa >= SA) { sa -= SA; pha ^= 1u; }
           }
         }
       }
@@ -448,7 +578,35 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         tc_fence_after();
         uint32_t acc = 0;
         for (int kb = kb0; kb < nkb; kb += kbs) {
-          {
+          if (kTmemA && halves) {
+            // Two halves: four MMAs each (K = 64), each after its own barrier;
+            // the first half's A columns are released while the second runs.
+            const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
+            const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * 64);
+            if (!wait_x(full_a(2 * sa), pha)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              mma_ts(d_tmem, a0, b0, idesc, acc);
+              mma_ts(d_tmem, a0 + 8, b0 + 2, idesc, 1u);
+              mma_ts(d_tmem, a0 + 16, b0 + 4, idesc, 1u);
+              mma_ts(d_tmem, a0 + 24, b0 + 6, idesc, 1u);
+              commit(a_free(2 * sa));
+            }
+            __syncwarp();
+            if (!wait_x(full_a(2 * sa + 1), pha)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+              const uint64_t b1 = b0 + (b_chunk >> 4);
+              mma_ts(d_tmem, a0 + 32, b1, idesc, 1u);
+              mma_ts(d_tmem, a0 + 40, b1 + 2, idesc, 1u);
+              mma_ts(d_tmem, a0 + 48, b1 + 4, idesc, 1u);
+              mma_ts(d_tmem, a0 + 56, b1 + 6, idesc, 1u);
+              commit(a_free(2 * sa + 1));
+              commit(empty(st));
+            }
+            __syncwarp();
+            acc = 1u;
+          } else {
             if (!wait_x(full_a(sa), pha)) { ok = false; break; }
             tc_fence_after();
             const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
@@ -540,9 +698,6 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         sa += kLanes;
         if (sa >= SA) { sa -= SA; pha ^= 1u; }
         if (!mbar_wait(full_tma(cur), cur_ph, abort_flag)) { ok = false; break; }
-        // Forward: the A stage must have been released by the MMAs of the
-        // fill that used it SA fills ago.
-        if (kTmemA && !mbar_wait(a_free(cur_a), cur_pha ^ 1u, abort_flag)) { ok = false; break; }
         const uint32_t wq = W_at(cur);
         const uint32_t sc = S_at(cur);
         if constexpr (MODE == kModeFwd) {
@@ -552,30 +707,46 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           const uint32_t sw = (src >> 1) & 3;
           const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a_col0 +
                                 static_cast<uint32_t>(cur_a * 64);
-          // The four 32-element groups of the fill; each is stored to tensor
-          // memory as soon as it is dequantized (16 columns, two BF16 per
-          // column, low half = even k), which keeps only 16 results live. A
-          // half past the reduction length (K % 128 == 64) is written as zeros,
-          // so neither the zero-filled codes nor a foreign scale can reach the
-          // MMA.
+          // The A stage (or, with halves, each half of it) must have been
+          // released by the MMAs of the fill that used it SA fills ago. A
+          // warp covers the fill's four 32-element groups (one warp per lane
+          // quarter) or two of them (one half); with halves it hands each
+          // half over on that half's barrier, else the whole fill at once.
+          // Each group is stored to tensor memory as soon as it is
+          // dequantized (16 columns, two BF16 per column, low half = even
+          // k), which keeps only 16 results live. A half past the reduction
+          // length (K % 128 == 64) is written as zeros, so neither the
+          // zero-filled codes nor a foreign scale can reach the MMA.
+          constexpr int kGroups = 4 / kParts;
+          const int units = (halves && kParts == 1) ? 2 : 1;
+          for (int u = 0; u < units && ok; ++u) {
+            const int half = (kParts == 2) ? hk : u;
+            const int jb = halves ? 2 * cur_a + half : cur_a;
+            if (!mbar_wait(a_free(jb), cur_pha ^ 1u, abort_flag)) { ok = false; break; }
 #pragma unroll
-          for (int cc = 0; cc < 4 / kParts; ++cc) {
-            const int c = hk * (4 / kParts) + cc;
-            uint32_t o[16];
-            if (kb_cur * kFillK + (c >> 1) * 64 >= p.R) {
+            for (int cc = 0; cc < kGroups; ++cc) {
+              const int c = hk * kGroups + cc;
+              if (units == 2 && (c >> 1) != half) continue;
+              uint32_t o[16];
+              if (kb_cur * kFillK + (c >> 1) * 64 >= p.R) {
 #pragma unroll
-              for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
-            } else {
-              const uint4 pk = lds128(prow + ((c ^ sw) << 4));
-              const uint32_t soff = c * 128 + src;
-              const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
-                                                                  : lds_u8(sc + soff);
-              dequant32<FMT>(pk, sbits, o);
+                for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
+              } else {
+                const uint4 pk = lds128(prow + ((c ^ sw) << 4));
+                const uint32_t soff = c * 128 + src;
+                const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
+                                                                    : lds_u8(sc + soff);
+                dequant32<FMT>(pk, sbits, o);
+              }
+              tmem_st_32x32b_x16(trow + static_cast<uint32_t>(c * 16), o);
             }
-            tmem_st_32x32b_x16(trow + static_cast<uint32_t>(c * 16), o);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            // (In a pair the odd CTA's relay thread passes this on.)
+            if (lane == 0) mbar_arrive(full_a(jb));
           }
-          tmem_wait_st();
-          tc_fence_before();
+          if (!ok) break;
         } else {
           // Thread = (reduction row r, feature half hf): 64 features = 2
           // groups, split over the kParts warps of the lane quarter. Packed
@@ -604,10 +775,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             }
           }
           fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full_a(cur_a));
         }
-        __syncwarp();
-        // (In a pair the odd CTA's relay thread passes this stage on.)
-        if (lane == 0) mbar_arrive(full_a(cur_a));
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -774,7 +944,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(acc_empty(0), 0));
+        if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(acc_empty(pipes ? (it & 1) : 0), 0));
         else mbar_arrive(acc_empty(pipes ? (it & 1) : 0));
       }
     }
@@ -794,11 +964,12 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
 
 }  // namespace
 
-template <int MODE, int FMT, int EPI, int LANES, int PAIR>
+template <int MODE, int FMT, int EPI, int LANES, int PAIR, int DQW>
 static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorMap& tw,
                                           const CUtensorMap& ts, const GemmArgs& p, int grid,
                                           size_t smem, cudaStream_t s) {
-  auto k = grouped_qgemm_kernel<MODE, FMT, EPI, LANES, PAIR>;
+  auto k = grouped_qgemm_kernel<MODE, FMT, EPI, LANES, PAIR, DQW>;
+  constexpr int kThreads = gemm_threads(DQW);
   // Raise the dynamic shared-memory limit once per (device, kernel) and, for
   // pairs, count the clusters that can be resident at once; later calls,
   // including ones under stream capture, skip both.
@@ -847,13 +1018,17 @@ static cudaError_t launch_grouped_qgemm_t(const CUtensorMap& tb, const CUtensorM
   }
 }
 
-cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, bool pair,
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_warps, bool pair,
                                  const CUtensorMap& tb, const CUtensorMap& tw,
                                  const CUtensorMap& ts, const GemmArgs& p, int grid, size_t smem,
                                  cudaStream_t s) {
-#define MOEQ_LANES(M_, F_, E_, P_)                                                          \
-  return lanes == 4 ? launch_grouped_qgemm_t<M_, F_, E_, 4, P_>(tb, tw, ts, p, grid, smem, s) \
-                    : launch_grouped_qgemm_t<M_, F_, E_, 2, P_>(tb, tw, ts, p, grid, smem, s);
+  // Eight dequant warps only with two lanes (one warp per lane quarter) and
+  // single CTAs.
+  if (dq_warps != 16 && !(dq_warps == 8 && lanes == 2 && !pair)) return cudaErrorInvalidValue;
+#define MOEQ_LANES(M_, F_, E_, P_)                                                               \
+  if (dq_warps == 8) return launch_grouped_qgemm_t<M_, F_, E_, 2, 0, 8>(tb, tw, ts, p, grid, smem, s); \
+  return lanes == 4 ? launch_grouped_qgemm_t<M_, F_, E_, 4, P_, 16>(tb, tw, ts, p, grid, smem, s) \
+                    : launch_grouped_qgemm_t<M_, F_, E_, 2, P_, 16>(tb, tw, ts, p, grid, smem, s);
 #define MOEQ_CASE(M_, F_, E_)                                                  \
   if (mode == M_ && fmt == F_ && epi == E_) {                                  \
     if (pair) { MOEQ_LANES(M_, F_, E_, 1) } else { MOEQ_LANES(M_, F_, E_, 0) } \
@@ -886,9 +1061,10 @@ uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair) {
 }
 
 uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E) {
-  // barriers, TMEM slot + abort flag (16 B), warp totals, tile list, epilogue
-  // staging (4 x 4 KiB, 128-byte aligned), alignment slack
-  return 8u * (2u * stages + 2u * a_stages + 5u) + 16u + 32u * 4u +
+  // barriers (two per A stage reserved for halves), TMEM slot + abort flag
+  // (16 B), warp totals, tile list, epilogue staging (4 x 4 KiB, 128-byte
+  // aligned), alignment slack
+  return 8u * (2u * stages + 4u * a_stages + 5u) + 16u + 32u * 4u +
          static_cast<uint32_t>(E + 1) * 4u + 128u + 4u * 4096u + 1024u;
 }
 

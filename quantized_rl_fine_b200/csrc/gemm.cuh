@@ -28,16 +28,21 @@ struct GemmArgs {
   int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages);
                               // multiple of the lane count
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
-  int32_t pipes;              // 1: two tile pipelines (two lanes, two issuers; not with pairs)
+  int32_t pipes;              // 1: two tile pipelines (two issuers, each accumulating whole tiles)
+  int32_t a_halves;           // forward: 1 = each A stage handed over in two 64-wide halves
   __nv_bfloat16* out;         // [M][ldo]
   int64_t ldo;
   __nv_bfloat16* saved;       // fwd SwiGLU: written [M][N]; bwd SwiGLU: read [M][2K]
+  // Forward with gathered token rows: row p of the GEMM input is
+  // b_src[b_rows[p]] ([*][R] BF16); NULL: the rows come from the tensor map.
+  const int32_t* b_rows;
+  const __nv_bfloat16* b_src;
 };
 
 // pair: forward only; a cluster of two CTAs per 256 output features with
 // M = 256 MMAs (BN a multiple of 32, an even number of feature tiles); the
 // grid is clamped to the pairs that can be resident together.
-cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, bool pair,
+cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_warps, bool pair,
                                  const CUtensorMap& tb, const CUtensorMap& tw,
                                  const CUtensorMap& ts, const GemmArgs& p, int grid, size_t smem,
                                  cudaStream_t s);
@@ -53,12 +58,12 @@ uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E);
 // so each stage is waited on by exactly one member of each role, which sees
 // every phase of the stage's barriers: a phase-parity wait can then never
 // mistake a phase two behind for the one it waits for.
+// The number of dequant warps (16, or 8 with two lanes) is a kernel template
+// parameter; the epilogue warpgroup follows them.
 constexpr int kProdWarps = 2;
 constexpr int kMaxIssuers = 2;
-constexpr int kDqWarps = 16;
 constexpr int kIssuerWarp0 = kProdWarps;
 constexpr int kDqWarp0 = kIssuerWarp0 + kMaxIssuers;
-constexpr int kEpiWarp0 = kDqWarp0 + kDqWarps;
-constexpr int kGemmThreads = 32 * (kEpiWarp0 + 4);
+constexpr int gemm_threads(int dq_warps) { return 32 * (kDqWarp0 + dq_warps + 4); }
 
 }  // namespace moeq

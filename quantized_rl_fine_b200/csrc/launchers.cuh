@@ -20,11 +20,14 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                          void* x_perm, int32_t* block_counts, cudaStream_t s);
 cudaError_t launch_combine(const void* rows, const int32_t* inv_perm, const float* gates, int T,
                            int k, int64_t D, void* out, int mode, cudaStream_t s);
-// out = x . R_e for the rows of each expert (forward adapter).
-cudaError_t launch_adapter_apply(const void* x, const void* R, const int32_t* offsets, int E,
-                                 int M, int K, void* out, cudaStream_t s);
-// dx = dxp . R_e^T and dR = sum over each expert's rows of x^T dxp, in one pass.
-cudaError_t launch_adapter_bwd(const void* x, const void* dxp, const void* R,
+// out = x . R_e for the rows of each expert (forward adapter); with rows (not
+// NULL), row p reads x[rows[p]].
+cudaError_t launch_adapter_apply(const void* x, const int32_t* rows, const void* R,
+                                 const int32_t* offsets, int E, int M, int K, void* out,
+                                 cudaStream_t s);
+// dx = dxp . R_e^T and dR = sum over each expert's rows of x^T dxp, in one pass;
+// with rows (not NULL), row p of x is x[rows[p]].
+cudaError_t launch_adapter_bwd(const void* x, const int32_t* rows, const void* dxp, const void* R,
                                const int32_t* offsets, int E, int K, void* dx, float* dR,
                                cudaStream_t s);
 // Expert parallelism: received rows, source-major <-> local expert-major

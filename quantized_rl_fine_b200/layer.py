@@ -5,6 +5,11 @@ forward : route_permute -> fwd GEMM (gate/up, SwiGLU [, adapter]) -> fwd GEMM
 backward: scatter (gate-scaled dy) -> bwd_dx down (SwiGLU backward) ->
           bwd_dx gate/up [+ adapter backward] -> combine (unpermute-sum)
 up-projection only: route_permute -> fwd GEMM (no epilogue)
+
+By default the permuted token rows are never written: routing returns the
+permutation only, and the gate/up GEMM (or, with the adapter, the adapter
+kernels) reads row p as x[perm_token[p]]. gather=False materializes x_perm in
+the routing call and feeds it to the GEMMs instead.
 """
 
 from __future__ import annotations
@@ -17,14 +22,15 @@ from .synth import QWeightT
 
 def forward(x: torch.Tensor, logits: torch.Tensor, w_gu: QWeightT, w_d: QWeightT, k: int,
             chunk_size: int, adapter: torch.Tensor | None = None, train: bool = False,
-            stream=None) -> dict:
+            stream=None, gather: bool = True) -> dict:
     T = x.shape[0]
-    r = M.moe_route_permute(logits, x, k, chunk_size, stream=stream)
-    h, saved = M.moe_grouped_qgemm_fwd(r.x_perm, w_gu, r, M.EPI_SWIGLU, adapter=adapter,
-                                       save_gu=train, stream=stream)
+    r = M.moe_route_permute(logits, None if gather else x, k, chunk_size, stream=stream)
+    a, a_rows = (x, r.perm_token) if gather else (r.x_perm, None)
+    h, saved = M.moe_grouped_qgemm_fwd(a, w_gu, r, M.EPI_SWIGLU, adapter=adapter,
+                                       save_gu=train, stream=stream, a_rows=a_rows)
     y_perm = M.moe_grouped_qgemm_fwd(h, w_d, r, M.EPI_NONE, stream=stream)
     y = M.moe_unpermute_combine(y_perm, r, r.gates, T, mode=0, stream=stream)
-    return dict(routing=r, h=h, saved_gu=saved, y_perm=y_perm, y=y)
+    return dict(routing=r, x=x, a=a, a_rows=a_rows, h=h, saved_gu=saved, y_perm=y_perm, y=y)
 
 
 def backward(state: dict, dy: torch.Tensor, w_gu: QWeightT, w_d: QWeightT,
@@ -36,7 +42,8 @@ def backward(state: dict, dy: torch.Tensor, w_gu: QWeightT, w_d: QWeightT,
                                      stream=stream)
     if adapter is not None:
         dx_perm, d_adapter = M.moe_grouped_qgemm_bwd_dx(dgu, w_gu, r, M.EPI_NONE, adapter=adapter,
-                                                        a=r.x_perm, stream=stream)
+                                                        a=state["a"], a_rows=state["a_rows"],
+                                                        stream=stream)
     else:
         dx_perm = M.moe_grouped_qgemm_bwd_dx(dgu, w_gu, r, M.EPI_NONE, stream=stream)
         d_adapter = None
@@ -45,7 +52,8 @@ def backward(state: dict, dy: torch.Tensor, w_gu: QWeightT, w_d: QWeightT,
 
 
 def up_projection(x: torch.Tensor, logits: torch.Tensor, w_up: QWeightT, k: int, chunk_size: int,
-                  stream=None) -> dict:
-    r = M.moe_route_permute(logits, x, k, chunk_size, stream=stream)
-    out = M.moe_grouped_qgemm_fwd(r.x_perm, w_up, r, M.EPI_NONE, stream=stream)
+                  stream=None, gather: bool = True) -> dict:
+    r = M.moe_route_permute(logits, None if gather else x, k, chunk_size, stream=stream)
+    a, a_rows = (x, r.perm_token) if gather else (r.x_perm, None)
+    out = M.moe_grouped_qgemm_fwd(a, w_up, r, M.EPI_NONE, stream=stream, a_rows=a_rows)
     return dict(routing=r, out=out)

@@ -70,11 +70,11 @@ def lib() -> ctypes.CDLL:
                                     vp, vp, vp, vp, sz, vp]
     L.moe_route_permute_noalloc.argtypes = [vp, vp, i64, i32, i32, i64, i32, vp, vp, vp, vp, vp,
                                             vp, vp, vp, vp, vp, vp]
-    L.moe_grouped_qgemm_fwd.argtypes = [vp, i64, ctypes.POINTER(QWeightC), ctypes.POINTER(GroupsC),
-                                        vp, i32, vp, vp, vp, sz, vp]
+    L.moe_grouped_qgemm_fwd.argtypes = [vp, vp, i64, ctypes.POINTER(QWeightC),
+                                        ctypes.POINTER(GroupsC), vp, i32, vp, vp, vp, sz, vp]
     L.moe_grouped_qgemm_bwd_dx.argtypes = [vp, i64, ctypes.POINTER(QWeightC),
                                            ctypes.POINTER(GroupsC), i32, vp, vp, vp, vp, vp, vp,
-                                           sz, vp]
+                                           vp, sz, vp]
     L.moe_unpermute_combine.argtypes = [vp, vp, vp, i64, i32, i64, vp, i32, vp]
     L.moe_get_device_error.argtypes = [ctypes.POINTER(i32), vp]
     L.moe_status_string.argtypes = [i32]
@@ -187,10 +187,11 @@ def qweight_c(w: QWeightT) -> QWeightC:
 def moe_grouped_qgemm_fwd(a: torch.Tensor, w: QWeightT, routing: Routing, epi: int = EPI_NONE,
                           adapter: torch.Tensor | None = None, save_gu: bool = False,
                           stream=None, out: torch.Tensor | None = None,
-                          saved: torch.Tensor | None = None):
-    """Returns out [M, N] (none) or (out [M, N/2], saved [M, N] or None) (swiglu)."""
-    _require_cuda(a, adapter)
-    M = a.shape[0]
+                          saved: torch.Tensor | None = None, a_rows: torch.Tensor | None = None):
+    """Returns out [M, N] (none) or (out [M, N/2], saved [M, N] or None) (swiglu).
+    With a_rows (int32 [M], e.g. routing.perm_token), row p of the input is a[a_rows[p]]."""
+    _require_cuda(a, adapter, a_rows)
+    M = a_rows.shape[0] if a_rows is not None else a.shape[0]
     F = w.N // 2 if epi == EPI_SWIGLU else w.N
     if out is None:
         out = torch.empty((M, F), dtype=torch.bfloat16, device=a.device)
@@ -199,8 +200,8 @@ def moe_grouped_qgemm_fwd(a: torch.Tensor, w: QWeightT, routing: Routing, epi: i
     qw, g = qweight_c(w), routing.groups()
     wsb = ctypes.c_size_t(0)
     L = lib()
-    args = lambda ws, wsz: (_p(a), M, ctypes.byref(qw), ctypes.byref(g), _p(adapter), epi,
-                            _p(out), _p(saved) if save_gu else None, ws, wsz, _stream(stream))
+    args = lambda ws, wsz: (_p(a), _p(a_rows), M, ctypes.byref(qw), ctypes.byref(g), _p(adapter),
+                            epi, _p(out), _p(saved) if save_gu else None, ws, wsz, _stream(stream))
     _check(L.moe_grouped_qgemm_fwd(*args(None, ctypes.byref(wsb))),
            "moe_grouped_qgemm_fwd (workspace query)")
     ws, wsp, wsz = _workspace(wsb.value, a.device)
@@ -213,9 +214,11 @@ def moe_grouped_qgemm_fwd(a: torch.Tensor, w: QWeightT, routing: Routing, epi: i
 def moe_grouped_qgemm_bwd_dx(dout: torch.Tensor, w: QWeightT, routing: Routing,
                              epi: int = EPI_NONE, saved_gu: torch.Tensor | None = None,
                              adapter: torch.Tensor | None = None, a: torch.Tensor | None = None,
-                             stream=None, out: torch.Tensor | None = None):
-    """Returns din ([M, K], or [M, 2K] for swiglu_bwd), plus d_adapter when an adapter is given."""
-    _require_cuda(dout, saved_gu, adapter, a)
+                             stream=None, out: torch.Tensor | None = None,
+                             a_rows: torch.Tensor | None = None):
+    """Returns din ([M, K], or [M, 2K] for swiglu_bwd), plus d_adapter when an adapter is given.
+    With a_rows, row p of the adapter's input a is a[a_rows[p]]."""
+    _require_cuda(dout, saved_gu, adapter, a, a_rows)
     M = dout.shape[0]
     width = 2 * w.K if epi == EPI_SWIGLU_BWD else w.K
     if out is None:
@@ -227,7 +230,8 @@ def moe_grouped_qgemm_bwd_dx(dout: torch.Tensor, w: QWeightT, routing: Routing,
     wsb = ctypes.c_size_t(0)
     L = lib()
     args = lambda ws, wsz: (_p(dout), M, ctypes.byref(qw), ctypes.byref(g), epi, _p(saved_gu),
-                            _p(adapter), _p(a), _p(out), _p(d_adapter), ws, wsz, _stream(stream))
+                            _p(adapter), _p(a), _p(a_rows), _p(out), _p(d_adapter), ws, wsz,
+                            _stream(stream))
     _check(L.moe_grouped_qgemm_bwd_dx(*args(None, ctypes.byref(wsb))),
            "moe_grouped_qgemm_bwd_dx (workspace query)")
     ws, wsp, wsz = _workspace(wsb.value, dout.device)

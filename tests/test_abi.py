@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.moe_abi_version() == 1
+    assert L.moe_abi_version() == 2
     assert L.moe_status_string(0) == b"MOE_OK"
     assert L.moe_status_string(4) == b"MOE_ERR_WORKSPACE"
 
@@ -49,11 +49,11 @@ def _groups(E=4):
 
 
 def _fwd(L, a=0x80000, M=64, qw=None, g=None, adapter=None, epi=0, out=0x90000, saved=None,
-         ws=None, wsb=None):
+         ws=None, wsb=None, rows=None):
     qw = qw or _qw()
     g = g or _groups(qw.E)
     wsb = wsb if wsb is not None else ctypes.c_size_t(0)
-    return L.moe_grouped_qgemm_fwd(a, M, ctypes.byref(qw), ctypes.byref(g), adapter, epi, out,
+    return L.moe_grouped_qgemm_fwd(a, rows, M, ctypes.byref(qw), ctypes.byref(g), adapter, epi, out,
                                    saved, ws, ctypes.byref(wsb), None)
 
 
@@ -85,19 +85,22 @@ def test_fwd_workspace_query_and_validation(L):
     assert _fwd(L, adapter=0xA0000, ws=0x100000, wsb=ok, a=0x80004) == 2
     # no workspace at all: fine without an adapter, an error with one
     qw, g = _qw(), _groups()
-    assert L.moe_grouped_qgemm_fwd(0x80004, 64, ctypes.byref(qw), ctypes.byref(g), None, 0,
+    assert L.moe_grouped_qgemm_fwd(0x80004, None, 64, ctypes.byref(qw), ctypes.byref(g), None, 0,
                                    0x90000, None, None, None, None) == 2
-    assert L.moe_grouped_qgemm_fwd(0x80000, 64, ctypes.byref(qw), ctypes.byref(g), 0xA0000, 0,
+    assert L.moe_grouped_qgemm_fwd(0x80000, None, 64, ctypes.byref(qw), ctypes.byref(g), 0xA0000, 0,
                                    0x90000, None, None, None, None) == 4
+    # a row index for gathered input rows: 16-byte aligned like every pointer
+    assert L.moe_grouped_qgemm_fwd(0x80000, 0xB0004, 64, ctypes.byref(qw), ctypes.byref(g), None, 0,
+                                   0x90000, None, None, None, None) == 2
 
 
 def test_bwd_argument_rules(L):
     qw, g = _qw(), _groups()
     wsb = ctypes.c_size_t(0)
 
-    def call(epi=0, saved=None, adapter=None, a=None, dad=None):
+    def call(epi=0, saved=None, adapter=None, a=None, dad=None, rows=None):
         return L.moe_grouped_qgemm_bwd_dx(0x80000, 64, ctypes.byref(qw), ctypes.byref(g), epi,
-                                          saved, adapter, a, 0x90000, dad, None,
+                                          saved, adapter, a, rows, 0x90000, dad, None,
                                           ctypes.byref(wsb), None)
     assert call() == moeq.MOE_OK
     assert call(epi=2) == 1                      # SwiGLU backward needs saved g|u
@@ -106,6 +109,8 @@ def test_bwd_argument_rules(L):
     assert call(adapter=0xA0000, a=0xC0000, dad=0xD0000) == moeq.MOE_OK
     assert call(epi=2, saved=0xB0000, adapter=0xA0000, a=0xC0000, dad=0xD0000) == 1
     assert call(a=0xC0000) == 1
+    assert call(rows=0xE0000) == 1               # a row index only with an adapter
+    assert call(adapter=0xA0000, a=0xC0000, dad=0xD0000, rows=0xE0000) == moeq.MOE_OK
     assert call(epi=1) == 1
 
 

@@ -77,10 +77,11 @@ def _check_routing_full(r, x, topk, gates, g, rows):
     assert np.array_equal(r.chunk_offsets.cpu().numpy()[:nch + 1], g.chunk_offsets)
     assert np.array_equal(r.perm_token.cpu().numpy(), g.perm_token)
     assert np.array_equal(r.inv_perm.cpu().numpy(), g.inv_perm)
-    idx = torch.as_tensor(rows, device=r.x_perm.device)
-    xp = bf16_bits(r.x_perm.index_select(0, idx))
-    xs = bf16_bits(x.index_select(0, torch.as_tensor(g.perm_token[rows], device=x.device)))
-    assert np.array_equal(xp, xs)
+    if r.x_perm is not None:
+        idx = torch.as_tensor(rows, device=r.x_perm.device)
+        xp = bf16_bits(r.x_perm.index_select(0, idx))
+        xs = bf16_bits(x.index_select(0, torch.as_tensor(g.perm_token[rows], device=x.device)))
+        assert np.array_equal(xp, xs)
 
 
 def _sample_experts(g, seed):
@@ -287,7 +288,8 @@ def _every_tile_forward(cfg, wl, st, g, R):
     dn_cols = _quarter_features(d // 128, 128)
     w_gu = _row_weights(wl["w_gu"], act, {e: np.concatenate([gu_feat[e], f + gu_feat[e]]) for e in act})
     w_d = _row_weights(wl["w_d"], act, {e: dn_cols for e in act})
-    x_perm = st["routing"].x_perm.cpu()
+    # the GEMM's input rows: x[perm_token] (the layer gathers them in the kernels)
+    x_perm = wl["x"].cpu()[torch.as_tensor(g.perm_token)]
     h_all, yp_all, sv_all = _rows_host(st["h"]), _rows_host(st["y_perm"]), _rows_host(st["saved_gu"])
     errs = {k: _Errors(k) for k in ("h", "y_perm", "saved_gu")}
     M = x_perm.shape[0]
@@ -330,7 +332,7 @@ def _every_tile_backward(cfg, wl, st, bw, g, R):
     w_gu = _col_weights(wl["w_gu"], act, {e: gu_groups for e in act})
     dyp_all, sv_all = bw["dy_perm"].cpu(), st["saved_gu"].cpu()
     dgu_all, dxp_all = bw["dgu"].cpu(), bw["dx_perm"].cpu()
-    x_perm = st["routing"].x_perm.cpu()
+    x_perm = wl["x"].cpu()[torch.as_tensor(g.perm_token)]
     Rsel = None if R is None else R[:, gu_groups]                   # [E][ng][32][32]
     dR_lib = None
     if R is not None:

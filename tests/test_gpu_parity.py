@@ -98,7 +98,7 @@ def _check_routing(r: moeq.Routing, logits, x, k, C, E):
     assert np.array_equal(r.chunk_offsets.cpu().numpy()[:nch + 1], g.chunk_offsets)
     assert np.array_equal(r.perm_token.cpu().numpy(), g.perm_token)
     assert np.array_equal(r.inv_perm.cpu().numpy(), g.inv_perm)
-    if x is not None:
+    if x is not None and r.x_perm is not None:
         xp = r.x_perm.cpu().view(torch.int16).numpy()
         assert np.array_equal(xp, x.cpu().view(torch.int16).numpy()[g.perm_token])
     return g
@@ -181,12 +181,12 @@ def _oracle_weights(wl):
     return out
 
 
-def _run_layer_and_compare(cfg, T=None):
+def _run_layer_and_compare(cfg, T=None, gather=True):
     wl = _gpu_workload(cfg, T)
     ow = _oracle_weights(wl)
     R = f64(wl["adapter"]) if cfg.adapter else None
     st = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], cfg.k, cfg.chunk_size,
-                       adapter=wl.get("adapter"), train=cfg.train)
+                       adapter=wl.get("adapter"), train=cfg.train, gather=gather)
     torch.cuda.synchronize()
     ref = O.moe_forward(f64(wl["x"]), wl["logits"].cpu().numpy(), cfg.k, cfg.chunk_size,
                         ow["w_gu"], ow["w_d"], R=R)
@@ -216,16 +216,45 @@ def _run_layer_and_compare(cfg, T=None):
     return st
 
 
-def test_tiny_int4_layer_forward():
-    _run_layer_and_compare(TINY_INT4)
+@pytest.mark.parametrize("gather", [True, False], ids=["gathered_rows", "x_perm"])
+def test_tiny_int4_layer_forward(gather):
+    _run_layer_and_compare(TINY_INT4, gather=gather)
 
 
-def test_tiny_train_forward_backward_with_adapter():
-    _run_layer_and_compare(TINY_TRAIN)
+@pytest.mark.parametrize("gather", [True, False], ids=["gathered_rows", "x_perm"])
+def test_tiny_train_forward_backward_with_adapter(gather):
+    _run_layer_and_compare(TINY_TRAIN, gather=gather)
 
 
-def test_ragged_mxfp4_train_with_adapter():
-    _run_layer_and_compare(RAGGED_MX)
+@pytest.mark.parametrize("gather", [True, False], ids=["gathered_rows", "x_perm"])
+def test_ragged_mxfp4_train_with_adapter(gather):
+    _run_layer_and_compare(RAGGED_MX, gather=gather)
+
+
+@pytest.mark.parametrize("cfg", [TINY_INT4, TINY_TRAIN, RAGGED_MX, MXFP4_UP],
+                         ids=["int4", "int4_train_adapter", "mxfp4_ragged", "mxfp4_up"])
+def test_gathered_rows_give_the_bits_of_materialized_rows(cfg):
+    """Reading row p as x[perm_token[p]] inside the kernels (no x_perm) and
+    reading a materialized x_perm give bit-identical outputs, forward and
+    backward."""
+    wl = _gpu_workload(cfg)
+    outs = []
+    for gather in (True, False):
+        if not cfg.swiglu:
+            st = layer.up_projection(wl["x"], wl["logits"], wl["w_up"], cfg.k, cfg.chunk_size,
+                                     gather=gather)
+            outs.append((st["out"].clone(),))
+            continue
+        st = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], cfg.k, cfg.chunk_size,
+                           adapter=wl.get("adapter"), train=cfg.train, gather=gather)
+        o = [st["y"].clone(), st["h"].clone()]
+        if cfg.train:
+            bw = layer.backward(st, wl["dy"], wl["w_gu"], wl["w_d"], adapter=wl.get("adapter"))
+            o += [bw["dx"].clone()] + ([bw["d_adapter"].clone()] if cfg.adapter else [])
+        outs.append(tuple(o))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
 
 
 def test_single_token():
@@ -257,7 +286,7 @@ def test_mxfp4_up_projection_full_size():
     """The bench workload at its full size: every output compared with the oracle."""
     cfg = MXFP4_UP
     wl = _gpu_workload(cfg)
-    st = layer.up_projection(wl["x"], wl["logits"], wl["w_up"], cfg.k, cfg.chunk_size)
+    st = layer.up_projection(wl["x"], wl["logits"], wl["w_up"], cfg.k, cfg.chunk_size, gather=False)
     torch.cuda.synchronize()
     ref = O.up_projection(f64(wl["x"]), wl["logits"].cpu().numpy(), cfg.k, cfg.chunk_size,
                           oracle_qweight(wl["w_up"]))
@@ -284,25 +313,44 @@ def test_each_lane_count_and_tile_width_matches_the_oracle(monkeypatch, cfg, lan
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
 
 
-@pytest.mark.parametrize("bn", [None, "192"], ids=["planned", "forced192"])
+@pytest.mark.parametrize("bn", [None, "176", "192"], ids=["planned", "forced176", "forced192"])
 def test_wide_token_tiles_match_the_oracle(monkeypatch, bn):
     """Token tiles wider than 96 rows: planned for the backward at about 150
     rows per expert, and forced for both directions (the forward then runs
-    with one MMA-issuing warp, as two 192-column partials and four A stages
-    do not fit tensor memory)."""
+    two tile pipelines with two A stages handed over in halves, as two
+    accumulators of more than 128 columns leave room for only two)."""
     if bn is not None:
         monkeypatch.setenv("MOEQ_BN", bn)
     _run_layer_and_compare(WIDE)
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
 
 
+@pytest.mark.parametrize("env", [{"MOEQ_HALVES": "1"}, {"MOEQ_HALVES": "1", "MOEQ_LANES": "4"},
+                                 {"MOEQ_HALVES": "1", "MOEQ_PIPES": "0"}, {"MOEQ_DQW": "8"},
+                                 {"MOEQ_DQW": "8", "MOEQ_HALVES": "1"}],
+                         ids=["halves", "halves_4lanes", "halves_nopipes", "dqw8", "dqw8_halves"])
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, RAGGED_MX], ids=["int4", "mxfp4_ragged"])
+def test_a_stage_halves_and_dequant_warp_counts_match_the_oracle(monkeypatch, cfg, env):
+    """The forward A stages handed over in 64-wide halves (two barriers per
+    stage), with two or four lanes and with or without tile pipelines, and the
+    eight-dequant-warp kernels, against the oracle (K % 128 == 64 tail
+    included)."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("pipes", ["1", "0"], ids=["pipelines", "one_issuer"])
 @pytest.mark.parametrize("cfg", [TINY_TRAIN, WIDE], ids=["int4", "wide_int4"])
-def test_cta_pair_forward_matches_the_oracle(monkeypatch, cfg):
-    """The opt-in CTA-pair forward kernels (clusters of two CTAs, M = 256
-    MMAs issued by the even CTA, each CTA holding half of the token rows)
-    against the oracle; both shapes have an even number of feature tiles in
-    both forward GEMMs, so every forward launch runs on pairs."""
+def test_cta_pair_forward_matches_the_oracle(monkeypatch, cfg, pipes):
+    """The CTA-pair forward kernels (clusters of two CTAs, M = 256 MMAs issued
+    by the even CTA, each CTA holding half of the token rows), with two tile
+    pipelines (and, at 192-row tiles, A stages handed over in halves) or one
+    issuer, against the oracle; both shapes have an even number of feature
+    tiles in both forward GEMMs, so every forward launch runs on pairs."""
     monkeypatch.setenv("MOEQ_PAIR", "1")
+    monkeypatch.setenv("MOEQ_PIPES", pipes)
     _run_layer_and_compare(cfg)
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
 
