@@ -396,12 +396,12 @@ def _step_fn(cfg, chunk):
 
 
 def _launches_per_step(cfg):
-    # routing: top-k and the single-pass tail for launches of at most 1024
-    # tokens whose token-by-expert bit matrix fits 8192 words; else top-k,
-    # scan and scatter. The permuted rows are not copied: the gate/up GEMM
-    # (or the adapter) gathers them.
+    # routing: top-k and the single-pass tail (which also copies the rows) for
+    # launches of at most 1024 tokens whose token-by-expert bit matrix fits
+    # 8192 words; else top-k, scan, scatter and, without the adapter, the row
+    # copy (with the adapter the adapter kernels gather the rows instead).
     words = (cfg.T + 31) // 32
-    route = 2 if words <= 32 and words * cfg.E <= 8192 else 3
+    route = 2 if words <= 32 and words * cfg.E <= 8192 else (3 if cfg.adapter else 4)
     if not cfg.swiglu:
         return route + 1
     n = route + 2 + 1                           # gate/up, down, combine
@@ -512,14 +512,14 @@ def run_ours(args, cfg):
         r = st["routing"]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            # the layer's call: row p of the input is x[perm_token[p]]
+            # the layer's own call (its input rows: x_perm, or x through perm_token)
             if not cfg.swiglu:
-                moeq.moe_grouped_qgemm_fwd(wl["x"], wl["w_up"], r, moeq.EPI_NONE,
-                                           a_rows=r.perm_token)
+                moeq.moe_grouped_qgemm_fwd(st["a"], wl["w_up"], r, moeq.EPI_NONE,
+                                           a_rows=st["a_rows"])
             else:
-                moeq.moe_grouped_qgemm_fwd(wl["x"], wl["w_gu"], r, moeq.EPI_SWIGLU,
+                moeq.moe_grouped_qgemm_fwd(st["a"], wl["w_gu"], r, moeq.EPI_SWIGLU,
                                            adapter=wl.get("adapter"), save_gu=cfg.train,
-                                           a_rows=r.perm_token)
+                                           a_rows=st["a_rows"])
         gemm_graphs.append(g)
     for i in range(max(3, args.warmup)):
         gemm_graphs[i % ROTATE].replay()
@@ -699,14 +699,12 @@ def run_prior_art(args, cfg):
         h = torch.empty((M, cfg.f), dtype=torch.bfloat16, device=dev)
         y = torch.empty((M, cfg.d if cfg.swiglu else cfg.f), dtype=torch.bfloat16, device=dev)
 
-        def fused():   # the layer's calls: rows gathered from x in the kernel
+        def fused():   # the layer's calls (no adapter: the permuted rows)
             if cfg.swiglu:
-                moeq.moe_grouped_qgemm_fwd(wl["x"], w_first, r, moeq.EPI_SWIGLU, out=h,
-                                           a_rows=r.perm_token)
+                moeq.moe_grouped_qgemm_fwd(r.x_perm, w_first, r, moeq.EPI_SWIGLU, out=h)
                 moeq.moe_grouped_qgemm_fwd(h, wl["w_d"], r, moeq.EPI_NONE, out=y)
             else:
-                moeq.moe_grouped_qgemm_fwd(wl["x"], w_first, r, moeq.EPI_NONE, out=y,
-                                           a_rows=r.perm_token)
+                moeq.moe_grouped_qgemm_fwd(r.x_perm, w_first, r, moeq.EPI_NONE, out=y)
         got = {}
 
         def prior():

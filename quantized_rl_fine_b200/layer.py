@@ -6,10 +6,13 @@ backward: scatter (gate-scaled dy) -> bwd_dx down (SwiGLU backward) ->
           bwd_dx gate/up [+ adapter backward] -> combine (unpermute-sum)
 up-projection only: route_permute -> fwd GEMM (no epilogue)
 
-By default the permuted token rows are never written: routing returns the
-permutation only, and the gate/up GEMM (or, with the adapter, the adapter
-kernels) reads row p as x[perm_token[p]]. gather=False materializes x_perm in
-the routing call and feeds it to the GEMMs instead.
+With the adapter the permuted token rows are never written: routing returns
+the permutation only and the adapter kernels read row p as x[perm_token[p]]
+(plain loads, at no extra cost). Without it the routing call writes x_perm
+and the gate/up GEMM reads it through its tensor map; gather=True makes the
+GEMM gather the rows itself instead (same bits; at 341 rows per expert on
+B200 its gathering producer is about 2.2x slower than the tensor-map copy,
+because each stage is handed over only once its row copies have landed).
 """
 
 from __future__ import annotations
@@ -22,8 +25,10 @@ from .synth import QWeightT
 
 def forward(x: torch.Tensor, logits: torch.Tensor, w_gu: QWeightT, w_d: QWeightT, k: int,
             chunk_size: int, adapter: torch.Tensor | None = None, train: bool = False,
-            stream=None, gather: bool = True) -> dict:
+            stream=None, gather: bool | None = None) -> dict:
     T = x.shape[0]
+    if gather is None:
+        gather = adapter is not None
     r = M.moe_route_permute(logits, None if gather else x, k, chunk_size, stream=stream)
     a, a_rows = (x, r.perm_token) if gather else (r.x_perm, None)
     h, saved = M.moe_grouped_qgemm_fwd(a, w_gu, r, M.EPI_SWIGLU, adapter=adapter,
@@ -52,8 +57,8 @@ def backward(state: dict, dy: torch.Tensor, w_gu: QWeightT, w_d: QWeightT,
 
 
 def up_projection(x: torch.Tensor, logits: torch.Tensor, w_up: QWeightT, k: int, chunk_size: int,
-                  stream=None, gather: bool = True) -> dict:
+                  stream=None, gather: bool = False) -> dict:
     r = M.moe_route_permute(logits, None if gather else x, k, chunk_size, stream=stream)
     a, a_rows = (x, r.perm_token) if gather else (r.x_perm, None)
     out = M.moe_grouped_qgemm_fwd(a, w_up, r, M.EPI_NONE, stream=stream, a_rows=a_rows)
-    return dict(routing=r, out=out)
+    return dict(routing=r, a=a, a_rows=a_rows, out=out)

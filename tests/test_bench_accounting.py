@@ -64,12 +64,12 @@ def test_step_accounting_of_a_training_step_with_adapter():
 
 
 @pytest.mark.parametrize("cfg,kernels", [
-    # top-k, routing tail (offsets, permutation), up GEMM (gathers the rows)
+    # top-k, routing tail (offsets, permutation, row copy), up GEMM
     (C.MXFP4_UP, 3),
     # top-k, tail, gate/up, down, combine
     (C.TRILLION_INT4.with_(T=128), 5),
-    # top-k, scan, scatter, gate/up, down, combine
-    (C.TRILLION_INT4.with_(T=2048), 6),
+    # top-k, scan, scatter, row copy, gate/up, down, combine
+    (C.TRILLION_INT4.with_(T=2048), 7),
     # routing (3), adapter (gathers the rows), gate/up, down, combine, scatter
     # of dy, two backward GEMMs, fused adapter backward, combine of dx
     (C.TRAIN_INT4, 12),

@@ -288,7 +288,7 @@ def _every_tile_forward(cfg, wl, st, g, R):
     dn_cols = _quarter_features(d // 128, 128)
     w_gu = _row_weights(wl["w_gu"], act, {e: np.concatenate([gu_feat[e], f + gu_feat[e]]) for e in act})
     w_d = _row_weights(wl["w_d"], act, {e: dn_cols for e in act})
-    # the GEMM's input rows: x[perm_token] (the layer gathers them in the kernels)
+    # the GEMM's input rows: x[perm_token] (x_perm, or gathered in the kernels)
     x_perm = wl["x"].cpu()[torch.as_tensor(g.perm_token)]
     h_all, yp_all, sv_all = _rows_host(st["h"]), _rows_host(st["y_perm"]), _rows_host(st["saved_gu"])
     errs = {k: _Errors(k) for k in ("h", "y_perm", "saved_gu")}

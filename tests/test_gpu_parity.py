@@ -181,7 +181,7 @@ def _oracle_weights(wl):
     return out
 
 
-def _run_layer_and_compare(cfg, T=None, gather=True):
+def _run_layer_and_compare(cfg, T=None, gather=None):
     wl = _gpu_workload(cfg, T)
     ow = _oracle_weights(wl)
     R = f64(wl["adapter"]) if cfg.adapter else None
