@@ -77,6 +77,11 @@ def _workloads():
         E=48, T=2048, name="trillion_int4_E48_k8_d7168_f2048_T2048")
     w["train_int4_E48_T512"] = C.TRAIN_INT4.with_(
         E=48, T=512, name="train_int4_adapter_E48_k8_d7168_f2048_T512")
+    # Zipf-skewed MXFP4 routing with 64 experts and the same mean of 256 rows
+    # per expert as the E=256, T=8192 layer (the ranks' bias is the same, so
+    # the head experts hold a larger share of the rows): for a full capture.
+    w["zipf_mxfp4_E64_T2048"] = C.ZIPF_MXFP4.with_(
+        E=64, T=2048, name="zipf_mxfp4_E64_k8_d4096_f1536_T2048")
     return w
 
 

@@ -201,13 +201,6 @@ adapter_apply_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restr
 constexpr int kGradWarps = 8;     // column blocks per CTA of the gradient kernel (one warp each)
 constexpr int kGradRows = 32;     // rows staged per step
 
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
-                                              uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
 // Backward, fused: grid (E, ceil(K / 256)), 256 threads. Warp (e, b) walks the
 // rows of expert e in ascending order, 32 at a time: it stages the rows' x and
 // dx' columns of block b in shared memory and from them forms both

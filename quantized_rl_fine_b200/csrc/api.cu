@@ -239,14 +239,15 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   // latency of the weight stream.
   const int avail = max_smem_optin();
   auto fits = [&](int s, int sa) {
-    return static_cast<int>(s * pl.stage_bytes + gemm_fixed_smem_bytes(s, sa, w->E)) <= avail;
+    return static_cast<int>(s * pl.stage_bytes + gemm_fixed_smem_bytes(mode, s, sa, w->E)) <= avail;
   };
-  if (mode == kModeFwd) {
+  if (mode != kModeBwd) {
     // A stage of a 128-wide fill: 64 tensor-memory columns. The most issuers
     // that still leave four A stages; with two issuers and wide accumulators
     // (more than 128 columns each) two A stages, handed over in halves, so
     // that a pipeline's next fill is dequantized while its previous fill's
-    // second half is multiplied. MOEQ_HALVES=0/1 overrides (tuning).
+    // second half is multiplied (forward only). MOEQ_HALVES=0/1 overrides
+    // (tuning).
     int halves_env = -1;
     if (const char* env = getenv("MOEQ_HALVES")) halves_env = atoi(env) != 0 ? 1 : 0;
     bool pipes_allowed = true;
@@ -261,10 +262,10 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
       if (sa >= 4) {
         pl.n_issuers = ni;
         pl.a_stages = sa;
-        pl.halves = halves_env == 1;
+        pl.halves = halves_env == 1 && mode == kModeFwd;
         break;
       }
-      if (ni == 2 && sa >= 2 && halves_env != 0 && pipes_allowed) {
+      if (mode == kModeFwd && ni == 2 && sa >= 2 && halves_env != 0 && pipes_allowed) {
         pl.n_issuers = ni;
         pl.a_stages = sa;
         pl.halves = true;
@@ -302,7 +303,7 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   if (const char* env = getenv("MOEQ_PIPES")) pl.pipes = (atoi(env) != 0);
   pl.pipes = pl.pipes && pl.n_issuers == 2;
   const int stages = pl.stages;
-  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(stages, pl.a_stages, w->E);
+  pl.smem = stages * pl.stage_bytes + gemm_fixed_smem_bytes(mode, stages, pl.a_stages, w->E);
   const int64_t bound = static_cast<int64_t>(pl.pair ? pl.n_ftiles / 2 : pl.n_ftiles) *
                         (std::min<int64_t>(w->E, M) + (M + pl.BN - 1) / pl.BN);
   if (pl.pair)   // CTAs, two per pair tile; the launch clamps to the resident pairs
@@ -342,7 +343,7 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   const uint64_t esz = int4 ? 2 : 1;
   const CUtensorMapDataType sdt = int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t E = w->E, N = w->N, K = w->K;
-  const uint32_t chunks = (mode == kModeFwd) ? 2 : 1;      // 64-element K chunks per fill
+  const uint32_t chunks = (mode == kModeBwd) ? 1 : 2;      // 64-element K chunks per fill
   {  // token rows: [M][R] BF16 viewed as (64, M, R/64) -> smem [chunk][BN rows][64]
     const uint64_t dims[3] = {64, static_cast<uint64_t>(M), static_cast<uint64_t>(R) / 64};
     const uint64_t strides[2] = {static_cast<uint64_t>(R) * 2, 128};
@@ -376,12 +377,15 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
         !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
   } else {
+    // backward: one box is the fill's reduction rows n (64, or 128 with A in
+    // tensor memory) x the tile's 128 features (64 B); scales [4 groups][rows]
+    const uint32_t fill = (mode == kModeBwdT) ? 128 : 64;
     const uint64_t wd[3] = {K / 2, E * N, 1};
     const uint64_t ws[2] = {K / 2, E * N * (K / 2)};
-    const uint32_t wb[3] = {64, 64, 1};
+    const uint32_t wb[3] = {64, fill, 1};
     const uint64_t sd[3] = {N, E * (K / 32), 1};
     const uint64_t ss[2] = {N * esz, E * (K / 32) * N * esz};
-    const uint32_t sb[3] = {64, 4, 1};
+    const uint32_t sb[3] = {fill, 4, 1};
     if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb,
                      CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
@@ -601,7 +605,11 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
   if (with_adapter && (epi != MOE_EPI_NONE || !a || !d_adapter)) return MOE_ERR_INVALID_ARG;
   if (!with_adapter && (a || a_rows || d_adapter)) return MOE_ERR_INVALID_ARG;
   if (epi == MOE_EPI_SWIGLU_BWD && !saved_gu) return MOE_ERR_INVALID_ARG;
-  const GemmPlan pl = plan_gemm(kModeBwd, M, w, w->K, 128, w->fmt);
+  // A in tensor memory (128-wide fills, the dequantized rows transposed on
+  // the way) unless MOEQ_BWD_SMEM_A=1 asks for the shared-memory form (tuning).
+  int bmode = kModeBwdT;
+  if (const char* env = getenv("MOEQ_BWD_SMEM_A")) bmode = (atoi(env) == 1) ? kModeBwd : kModeBwdT;
+  const GemmPlan pl = plan_gemm(bmode, M, w, w->K, 128, w->fmt);
   const size_t need = with_adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
   if ((st = check_workspace(ws, ws_bytes, need)) != MOE_OK) return st;
   if (!ws && ws_bytes) return MOE_OK;   // size query
@@ -613,14 +621,14 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
     return MOE_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (epi == MOE_EPI_SWIGLU_BWD) {
-    return run_gemm(kModeBwd, epi, dout, M, w, g, din, 2 * static_cast<int64_t>(w->K),
+    return run_gemm(bmode, epi, dout, M, w, g, din, 2 * static_cast<int64_t>(w->K),
                     const_cast<void*>(saved_gu), pl, s);
   }
   if (!with_adapter) {
-    return run_gemm(kModeBwd, epi, dout, M, w, g, din, w->K, nullptr, pl, s);
+    return run_gemm(bmode, epi, dout, M, w, g, din, w->K, nullptr, pl, s);
   }
   void* dxa = ws;
-  st = run_gemm(kModeBwd, epi, dout, M, w, g, dxa, w->K, nullptr, pl, s);
+  st = run_gemm(bmode, epi, dout, M, w, g, dxa, w->K, nullptr, pl, s);
   if (st != MOE_OK) return st;
   return cuda_status(launch_adapter_bwd(a, a_rows, dxa, adapter, g->expert_offsets, w->E, w->K,
                                         din, d_adapter, s));

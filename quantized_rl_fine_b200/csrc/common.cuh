@@ -309,6 +309,29 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
       : "memory");
 }
 
+// Stores 16 lanes x 16 columns: thread t writes r[2j + i] to lane 8i + t/4,
+// column 4j + t%4 of the block at taddr (j < 4, i < 2). This is the fragment
+// layout ldmatrix gives (thread t: row t/4 of each 8 x 8 matrix, or with
+// .trans its column t/4), so matrices loaded with ldmatrix go to tensor
+// memory without a shuffle. taddr's lane must lie in the warp's quarter.
+__device__ __forceinline__ void tmem_st_16x128b_x4(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
+// Four 8 x 8 BF16 matrices from shared memory, transposed: thread t supplies
+// the address of row t % 8 of matrix t / 8 and receives, in register m, the
+// elements (row 2 (t%4), column t/4) (low half) and (row 2 (t%4) + 1,
+// column t/4) (high half) of matrix m.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "

@@ -17,10 +17,13 @@
 // B (N = BN):
 //
 //   forward  D[f, t] = sum_k W[e][f][k] * a[t][k]     (A K-major, in tensor memory)
-//   backward D[f, t] = sum_n W[e][n][f] * dout[t][n]  (A MN-major, in shared memory)
+//   backward D[f, t] = sum_n W[e][n][f] * dout[t][n]  (A K-major in tensor memory, the
+//                                                      dequantized rows transposed on
+//                                                      the way; or MN-major in shared
+//                                                      memory)
 //
-// The reduction is walked in fills of 128 (forward) or 64 (backward)
-// elements. Fill f of the CTA belongs to pipeline lane f % kLanes, whose
+// The reduction is walked in fills of 128 (A in tensor memory) or 64 (A in
+// shared memory) elements. Fill f of the CTA belongs to pipeline lane f % kLanes, whose
 // dequant group (four or eight warps covering the four tensor-memory lane
 // quarters) turns its packed codes into BF16 in registers and then into the A
 // stage; producer warp f % kProdWarps issues its copies (token rows, packed
@@ -53,6 +56,8 @@ static_assert(gemm_threads(16) <= 1024 && ((gemm_threads(16) / 32 + 3) / 4) * 32
               "roles must fit 80 registers a thread");
 constexpr int kTileF = 128;            // output features per tile (MMA M)
 constexpr uint32_t kABytes = kTileF * 64 * 2;   // 16 KiB dequantized A tile (backward fill)
+constexpr uint32_t kStageBytesEpi = 2048;       // epilogue staging block per warp
+constexpr uint32_t kScratchBytes = 1024;        // kModeBwdT transpose scratch per dequant warp
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -205,10 +210,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   constexpr int kWRound = PAIR ? 32 : 16;
   constexpr uint32_t kScEl = (FMT == MOE_W_INT4_G32_BF16) ? 2 : 1;
   constexpr bool kGluRows = (MODE == kModeFwd && EPI == MOE_EPI_SWIGLU);
-  // Forward: fills of 128 reduction elements; the dequantized A tile goes to
-  // tensor memory (two 32-column sub-stages per fill). Backward: fills of 64,
-  // A in a 128B-swizzled MN-major shared-memory tile.
-  constexpr bool kTmemA = (MODE == kModeFwd);
+  // Forward and kModeBwdT: fills of 128 reduction elements; the dequantized
+  // A tile goes to tensor memory (64 columns per fill). kModeBwd: fills of
+  // 64, A in a 128B-swizzled MN-major shared-memory tile.
+  constexpr bool kTmemA = (MODE != kModeBwd);
   constexpr int kFillK = kTmemA ? 128 : 64;
   constexpr uint32_t kSmemA = kTmemA ? 0u : kABytes;
   constexpr uint32_t kWqFill = kTmemA ? 8192u : 4096u;            // packed bytes per fill
@@ -255,8 +260,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* warp_tot = reinterpret_cast<int32_t*>(tmem_slot + 4);          // [32]
   int32_t* tile_start = warp_tot + 32;                                      // [E + 1]
-  // Epilogue staging: one 4 KiB block per epilogue warp (16 token rows x 64 BF16 used).
+  // Epilogue staging: one 2 KiB block per epilogue warp (16 token rows x 64
+  // BF16); then, for kModeBwdT, a 1 KiB transpose scratch per dequant warp.
   const uint32_t stg_base = (smem_u32(tile_start + p.E + 1) + 127u) & ~127u;
+  const uint32_t scratch_base = stg_base + 4u * kStageBytesEpi;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -747,6 +754,67 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             if (lane == 0) mbar_arrive(full_a(jb));
           }
           if (!ok) break;
+        } else if constexpr (MODE == kModeBwdT) {
+          // A in tensor memory, K-major: lane = output feature (k) of the
+          // tile, column = a pair of reduction rows (n, n + 1), low half n.
+          // A packed row runs along k, and the warp's lane quarter q holds
+          // exactly quantization group q of every row, so a lane dequantizes
+          // one row n (32 features) at a time. The warp stages its 32 rows
+          // in its scratch 16 features at a time ([32 rows][32 B]; chunk c of
+          // row r at c ^ ((r >> 2) & 1), conflict-free for these writes and
+          // for the reads) and reads them back transposed with ldmatrix: in
+          // its fragments thread t holds feature t / 4 and the row pair
+          // (2 (t%4), 2 (t%4) + 1), which is the register layout of the
+          // tcgen05.st 16x128b shape (lane t / 4, column t % 4). Packed rows
+          // are 64 bytes with the TMA 64-byte swizzle, scales [4 groups][128
+          // rows]; rows past the reduction length (N % 128 == 64) are zeros.
+          constexpr int kRowsPerWarp = kFillK / kParts;    // 64 or 128
+          const uint32_t scr = scratch_base + static_cast<uint32_t>(warp - kDqWarp0) * kScratchBytes;
+          const uint32_t wr = scr + static_cast<uint32_t>(lane) * 32u;
+          const uint32_t wsw = static_cast<uint32_t>(lane >> 2) & 1u;
+          // ldmatrix: lane l gives row l % 8 of matrix l / 8; the matrices are
+          // (rows 0-7, features 0-7), (rows 0-7, 8-15), (rows 8-15, 0-7),
+          // (rows 8-15, 8-15), i.e. registers (lane, column) blocks (0, 0),
+          // (8, 0), (0, 4), (8, 4) of the 16x128b store.
+          const int lm_row = (lane & 7) + ((lane >> 4) << 3);
+          const int lm_chunk = (lane >> 3) & 1;
+          const uint32_t lm0 = scr + static_cast<uint32_t>(lm_row) * 32u +
+                               (static_cast<uint32_t>(lm_chunk ^ ((lm_row >> 2) & 1)) << 4);
+          const uint32_t lm1 = lm0 + 16u * 32u;   // rows 16-31 (same swizzle)
+          if (!mbar_wait(a_free(cur_a), cur_pha ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t tstage = tmem_base + a_col0 + static_cast<uint32_t>(cur_a * 64);
+          for (int sj = 0; sj < kRowsPerWarp / 32; ++sj) {
+            const int nb = hk * kRowsPerWarp + sj * 32;     // first row of the 32
+            const int n = nb + lane;
+            uint32_t o[16];
+            if (kb_cur * kFillK + n >= p.R) {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
+            } else {
+              const uint4 pk = lds128(wq + n * 64 + ((q ^ ((n >> 1) & 3)) << 4));
+              const uint32_t soff = q * 128 + n;
+              const uint32_t sbits = (FMT == MOE_W_INT4_G32_BF16) ? lds_u16(sc + soff * 2)
+                                                                  : lds_u8(sc + soff);
+              dequant32<FMT>(pk, sbits, o);
+            }
+            const uint32_t tcol = tstage + static_cast<uint32_t>(nb >> 1);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // features 16h .. 16h + 15 of the 32 rows
+              sts128(wr + (wsw << 4), o[8 * h], o[8 * h + 1], o[8 * h + 2], o[8 * h + 3]);
+              sts128(wr + ((wsw ^ 1u) << 4), o[8 * h + 4], o[8 * h + 5], o[8 * h + 6], o[8 * h + 7]);
+              __syncwarp();
+              uint32_t tr[8];
+              ldsm_x4_trans(lm0, tr[0], tr[1], tr[2], tr[3]);
+              ldsm_x4_trans(lm1, tr[4], tr[5], tr[6], tr[7]);
+              tmem_st_16x128b_x4(tcol + (static_cast<uint32_t>(q * 32 + 16 * h) << 16), tr);
+              __syncwarp();
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full_a(cur_a));
         } else {
           // Thread = (reduction row r, feature half hf): 64 features = 2
           // groups, split over the kParts warps of the lane quarter. Packed
@@ -787,7 +855,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     // 16-byte stores, only for rows that belong to the tile's expert.
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int fr = q * 32 + lane;           // accumulator row = tile feature
-    const uint32_t stg = stg_base + static_cast<uint32_t>(q) * 4096u;
+    const uint32_t stg = stg_base + static_cast<uint32_t>(q) * kStageBytesEpi;
     uint16_t* stg_ptr = reinterpret_cast<uint16_t*>(gbase + (stg - base));
     static_assert(kMaxIssuers <= 3, "the epilogue sums at most three partial accumulators");
     int it = 0;
@@ -876,7 +944,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             }
           }
           __syncwarp();
-        } else if constexpr (MODE == kModeBwd && EPI == MOE_EPI_SWIGLU_BWD) {
+        } else if constexpr (MODE != kModeFwd && EPI == MOE_EPI_SWIGLU_BWD) {
           const int f = tl.ft * kTileF + fr;      // feature of dh (< K)
           const bool fok = f < p.F;
           // saved g of row (row0 + c0 + j) and feature f; its u is K further on
@@ -1044,6 +1112,10 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_w
   MOEQ_CASE_SINGLE(kModeBwd, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU_BWD)
   MOEQ_CASE_SINGLE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
   MOEQ_CASE_SINGLE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU_BWD)
+  MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
+  MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU_BWD)
+  MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
+  MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU_BWD)
 #undef MOEQ_CASE_SINGLE
 #undef MOEQ_CASE
 #undef MOEQ_LANES
@@ -1053,19 +1125,21 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_w
 uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair) {
   const uint32_t el = (fmt == MOE_W_INT4_G32_BF16) ? 2u : 1u;
   uint32_t b;
-  if (mode == kModeFwd)   // B 2 chunks (BN / 2 rows in a pair), packed 128 rows x 64 B, scales 4 x 128
+  if (mode != kModeBwd)   // B 2 chunks (BN / 2 rows in a pair), packed 128 rows x 64 B, scales 4 x 128
     b = static_cast<uint32_t>(pair ? BN / 2 : BN) * 256u + 8192u + 512u * el;
   else                    // B 1 chunk, A 16 KiB, packed 64 rows x 64 B, scales 4 x 64
     b = static_cast<uint32_t>(BN) * 128u + kABytes + 4096u + 256u * el;
   return (b + 1023u) & ~1023u;
 }
 
-uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E) {
+uint32_t gemm_fixed_smem_bytes(int mode, int stages, int a_stages, int E) {
   // barriers (two per A stage reserved for halves), TMEM slot + abort flag
-  // (16 B), warp totals, tile list, epilogue staging (4 x 4 KiB, 128-byte
-  // aligned), alignment slack
+  // (16 B), warp totals, tile list, epilogue staging (4 blocks, 128-byte
+  // aligned), the transpose scratch of kModeBwdT (16 dequant warps at most),
+  // alignment slack
   return 8u * (2u * stages + 4u * a_stages + 5u) + 16u + 32u * 4u +
-         static_cast<uint32_t>(E + 1) * 4u + 128u + 4u * 4096u + 1024u;
+         static_cast<uint32_t>(E + 1) * 4u + 128u + 4u * kStageBytesEpi +
+         (mode == kModeBwdT ? 16u * kScratchBytes : 0u) + 1024u;
 }
 
 }  // namespace moeq

@@ -8,8 +8,9 @@
 
 namespace moeq {
 
-constexpr int kModeFwd = 0;   // D[f, t] = sum_k W[e][f][k] a[t][k]
-constexpr int kModeBwd = 1;   // D[f, t] = sum_n W[e][n][f] dout[t][n]
+constexpr int kModeFwd = 0;    // D[f, t] = sum_k W[e][f][k] a[t][k]
+constexpr int kModeBwd = 1;    // D[f, t] = sum_n W[e][n][f] dout[t][n], A in shared memory
+constexpr int kModeBwdT = 2;   // the same, A in tensor memory (128-wide fills, transposed dequant)
 
 struct GemmArgs {
   const int32_t* offsets;     // [E+1] expert row offsets
@@ -25,7 +26,7 @@ struct GemmArgs {
   int32_t F;                  // output features (fwd: N or N/2 with SwiGLU; bwd: K)
   int32_t R;                  // reduction length (fwd: K; bwd: N)
   int32_t stages;             // shared-memory fills in flight (multiple of the lane count)
-  int32_t a_stages;           // A stages (forward: in tensor memory; backward: = stages);
+  int32_t a_stages;           // A stages (in tensor memory; shared-memory backward: = stages);
                               // multiple of the lane count
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
   int32_t pipes;              // 1: two tile pipelines (two issuers, each accumulating whole tiles)
@@ -47,7 +48,7 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_w
                                  const CUtensorMap& ts, const GemmArgs& p, int grid, size_t smem,
                                  cudaStream_t s);
 uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair);
-uint32_t gemm_fixed_smem_bytes(int stages, int a_stages, int E);
+uint32_t gemm_fixed_smem_bytes(int mode, int stages, int a_stages, int E);
 // Warp roles, in order: kProdWarps TMA producers, up to kMaxIssuers
 // MMA-issuing warps, kDqWarps dequant warps split into LANES groups (LANES is a
 // kernel template parameter, 2 or 4), one epilogue warpgroup. Fill f (the

@@ -365,3 +365,14 @@ def test_forward_without_tile_pipelines_matches_the_oracle(monkeypatch, cfg):
     monkeypatch.setenv("MOEQ_LANES", "2")
     _run_layer_and_compare(cfg)
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, RAGGED_MX, WIDE], ids=["int4", "mxfp4_ragged", "wide_int4"])
+def test_shared_memory_backward_matches_the_oracle(monkeypatch, cfg):
+    """The backward GEMMs keep their A operand in tensor memory by default
+    (128-wide fills, the dequantized rows transposed on the way); this runs
+    the shared-memory form (64-wide fills, MN-major A; 192-row tiles from 128
+    rows per expert on) against the oracle."""
+    monkeypatch.setenv("MOEQ_BWD_SMEM_A", "1")
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
