@@ -321,6 +321,12 @@ const char* moe_status_string(moe_status s);
 /* ABI revision of this header, for bindings to check. */
 int32_t moe_abi_version(void);
 
+/* 1 when the library was built with NVTX ranges (the default): every entry
+ * point that launches work opens a range named after itself for its
+ * duration on the host (a no-op unless a profiler is attached). 0 when built
+ * with -DMOEQ_NVTX=0. */
+int32_t moe_nvtx_enabled(void);
+
 /*
  * Test hooks (not on the hot path).
  *

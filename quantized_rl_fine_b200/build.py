@@ -49,7 +49,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     os.makedirs(LIB_DIR, exist_ok=True)
     tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-o", tmp, os.path.join(CSRC, "moeq_all.cu")]
+    flags = list(NVCC_FLAGS)
+    if os.environ.get("MOEQ_NVTX") == "0":   # build without NVTX ranges
+        flags.append("-DMOEQ_NVTX=0")
+    cmd = [_nvcc(), *flags, "-o", tmp, os.path.join(CSRC, "moeq_all.cu")]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

@@ -12,6 +12,27 @@
 #include "gemm.cuh"
 #include "launchers.cuh"
 
+// NVTX ranges around every entry point that launches work (header-only NVTX
+// v3: a no-op unless a profiler has injected its tool). Compiled out with
+// -DMOEQ_NVTX=0.
+#ifndef MOEQ_NVTX
+#define MOEQ_NVTX 1
+#endif
+#if MOEQ_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace moeq {
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+}  // namespace moeq
+#define MOEQ_TRACE(name) const ::moeq::TraceRange moeq_trace_range_(name)
+#else
+#define MOEQ_TRACE(name) ((void)0)
+#endif
+
 namespace moeq {
 
 
@@ -432,6 +453,8 @@ extern "C" {
 
 int32_t moe_abi_version(void) { return MOEQ_ABI_VERSION; }
 
+int32_t moe_nvtx_enabled(void) { return MOEQ_NVTX ? 1 : 0; }
+
 const char* moe_status_string(moe_status s) {
   switch (s) {
     case MOE_OK: return "MOE_OK";
@@ -451,6 +474,7 @@ moe_status moe_route_permute(const float* logits, const void* x, int64_t T, int3
                              int32_t* chunk_offsets, int32_t* num_chunks, int32_t* perm_token,
                              int32_t* inv_perm, void* x_perm, void* ws, size_t* ws_bytes,
                              void* stream) {
+  MOEQ_TRACE("moe_route_permute");
   if (T < 1 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || chunk_size < 1)
     return MOE_ERR_INVALID_ARG;
   if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
@@ -533,6 +557,7 @@ moe_status moe_route_permute_noalloc(const float* logits, const void* x, int64_t
                                      int32_t* num_active, int32_t* chunk_offsets,
                                      int32_t* num_chunks, int32_t* perm_token, int32_t* inv_perm,
                                      void* x_perm, void* stream) {
+  MOEQ_TRACE("moe_route_permute_noalloc");
   if (T < 1 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E || chunk_size < 1)
     return MOE_ERR_INVALID_ARG;
   if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
@@ -563,6 +588,7 @@ moe_status moe_grouped_qgemm_fwd(const void* a, const int32_t* a_rows, int64_t M
                                  const moe_qweight* w, const moe_groups* g, const void* adapter,
                                  int32_t epi, void* out, void* saved_gu, void* ws,
                                  size_t* ws_bytes, void* stream) {
+  MOEQ_TRACE("moe_grouped_qgemm_fwd");
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -597,6 +623,7 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
                                     const void* adapter, const void* a, const int32_t* a_rows,
                                     void* din, float* d_adapter, void* ws, size_t* ws_bytes,
                                     void* stream) {
+  MOEQ_TRACE("moe_grouped_qgemm_bwd_dx");
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (M < 1 || M >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -637,6 +664,7 @@ moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweig
 moe_status moe_unpermute_combine(const void* rows, const int32_t* inv_perm, const float* gates,
                                  int64_t T, int32_t k, int64_t D, void* out, int32_t mode,
                                  void* stream) {
+  MOEQ_TRACE("moe_unpermute_combine");
   if (!rows || !inv_perm || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || k < 1 || k > 32 || D < 8 || D % 8 != 0 || (mode != 0 && mode != 1))
     return MOE_ERR_INVALID_ARG;
@@ -669,6 +697,7 @@ moe_status moe_test_dequant(const void* packed, const void* scales, int64_t R, i
 
 moe_status moe_dequant_experts(const moe_qweight* w, const int32_t* experts, int32_t count,
                                void* out, void* stream) {
+  MOEQ_TRACE("moe_dequant_experts");
   moe_status st = check_qweight(w);
   if (st != MOE_OK) return st;
   if (!experts || !out || count < 0) return MOE_ERR_INVALID_ARG;
@@ -696,6 +725,7 @@ moe_status moe_ep_regroup(const int32_t* counts, int32_t W, int32_t E_loc, int64
                           int32_t chunk_size, int32_t* expert_offsets, int32_t* active,
                           int32_t* num_active, int32_t* chunk_offsets, int32_t* num_chunks,
                           void* stream) {
+  MOEQ_TRACE("moe_ep_regroup");
   if (!counts || W < 1 || E_loc < 1 || static_cast<int64_t>(W) * E_loc > ep_max_entries())
     return MOE_ERR_INVALID_ARG;
   if (R < 0 || R >= (int64_t(1) << 31) || D < 8 || D % 8 != 0) return MOE_ERR_INVALID_ARG;

@@ -32,7 +32,7 @@ DEVERR_NONE, DEVERR_WAIT_TIMEOUT, DEVERR_BAD_OFFSETS = 0, 1, 2
 EXPORTED = ("moe_route_permute", "moe_route_permute_noalloc", "moe_grouped_qgemm_fwd", "moe_grouped_qgemm_bwd_dx",
             "moe_unpermute_combine", "moe_get_device_error", "moe_status_string",
             "moe_abi_version", "moe_test_dequant", "moe_test_set_wait_budget",
-            "moe_dequant_experts", "moe_ep_regroup")
+            "moe_dequant_experts", "moe_ep_regroup", "moe_nvtx_enabled")
 
 
 class MoeError(RuntimeError):

@@ -36,6 +36,11 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_abi_version_and_status_strings(L):
     assert L.moe_abi_version() == 2
+
+
+def test_default_build_has_nvtx_ranges(L):
+    # every entry point that launches work opens an NVTX range (compile flag MOEQ_NVTX)
+    assert L.moe_nvtx_enabled() == 1
     assert L.moe_status_string(0) == b"MOE_OK"
     assert L.moe_status_string(4) == b"MOE_ERR_WORKSPACE"
 
