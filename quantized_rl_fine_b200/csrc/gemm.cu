@@ -858,10 +858,36 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     const uint32_t stg = stg_base + static_cast<uint32_t>(q) * kStageBytesEpi;
     uint16_t* stg_ptr = reinterpret_cast<uint16_t*>(gbase + (stg - base));
     static_assert(kMaxIssuers <= 3, "the epilogue sums at most three partial accumulators");
+    // SwiGLU backward: the saved g and u of 16 token rows x this warp's 32
+    // features come into the warp's staging block ([16 rows][32 g | 32 u],
+    // 2 KiB) by cp.async, 16 bytes a copy and four copies a lane, one chunk
+    // ahead: the first chunk of a tile before its accumulator is waited for,
+    // the next one as soon as the previous chunk has been written out. Rows
+    // past the tile are zero-filled; a warp whose features lie past F copies
+    // nothing.
+    constexpr bool kGuStaged = (MODE != kModeFwd && EPI == MOE_EPI_SWIGLU_BWD);
+    auto prefetch_gu = [&](const Tile& tl, int c0) {
+      const int fb = tl.ft * kTileF + q * 32;
+      if (fb >= p.F) return;
+      const int nrows = min(16, tl.row_end - (tl.row0 + c0));
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int idx = lane + 32 * j;
+        const int rr = idx >> 3, pc = idx & 7;          // row, 16-byte piece (4 of g, 4 of u)
+        const bool ok = rr < nrows;
+        const __nv_bfloat16* src =
+            p.saved + (ok ? static_cast<int64_t>(tl.row0 + c0 + rr) * (2 * K) + (pc < 4 ? 0 : K) +
+                                fb + (pc & 3) * 8
+                          : 0);
+        cp_async_16(stg + static_cast<uint32_t>(rr * 128 + pc * 16), src, ok ? 16u : 0u);
+      }
+      cp_async_commit();
+    };
     int it = 0;
     int r0 = 0;                             // (first fill of the tile) % NI
     for (int t = t_first; t < total; t += t_step, ++it) {
       const Tile tl = tile_at(t);
+      if constexpr (kGuStaged) prefetch_gu(tl, 0);
       // Issuer j wrote its partial in this tile iff one of the tile's nkb
       // fills f has f % NI == j. With tile pipelines the tile's whole sum is
       // in accumulator it % 2.
@@ -947,34 +973,22 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         } else if constexpr (MODE != kModeFwd && EPI == MOE_EPI_SWIGLU_BWD) {
           const int f = tl.ft * kTileF + fr;      // feature of dh (< K)
           const bool fok = f < p.F;
-          // saved g of row (row0 + c0 + j) and feature f; its u is K further on
-          const uint16_t* sv = reinterpret_cast<const uint16_t*>(p.saved) +
-                               static_cast<int64_t>(tl.row0 + c0) * (2 * K) + (fok ? f : 0);
-          // Staging row: [0,32) dg, [32,64) du of this warp's 32 features.
-          // Two rows at a time: their saved g and u are loaded first (no
-          // branch, so the loads are in flight together), then combined.
+          // This chunk's g and u have landed; each lane turns its own two
+          // slots of every row (g -> dg, u -> du) in place, so the block is
+          // then the [16 rows][32 dg | 32 du] staging of the output.
+          cp_async_wait<0>();
+          __syncwarp();
 #pragma unroll
-          for (int h8 = 0; h8 < 16; h8 += 2) {
-            uint16_t gb[2], ub[2];
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const bool ok = fok && (h8 + jj) < nrows;
-              const uint16_t* src = sv + (ok ? (h8 + jj) * (2 * K) : 0);
-              gb[jj] = ok ? __ldg(src) : uint16_t(0);
-              ub[jj] = ok ? __ldg(src + K) : uint16_t(0);
-            }
-#pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              const float g = __uint_as_float(static_cast<uint32_t>(gb[jj]) << 16);
-              const float u = __uint_as_float(static_cast<uint32_t>(ub[jj]) << 16);
-              const float s = sigmoid_f(g);
-              const float x = v[h8 + jj];
-              const bool ok = fok && (h8 + jj) < nrows;
-              const uint16_t dg = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(x * u * s * (1.0f + g * (1.0f - s)))) : uint16_t(0);
-              const uint16_t du = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(x * g * s)) : uint16_t(0);
-              stg_ptr[(h8 + jj) * 64 + lane] = dg;
-              stg_ptr[(h8 + jj) * 64 + 32 + lane] = du;
-            }
+          for (int jj = 0; jj < 16; ++jj) {
+            const bool ok = fok && jj < nrows;
+            const float g = __uint_as_float(static_cast<uint32_t>(stg_ptr[jj * 64 + lane]) << 16);
+            const float u = __uint_as_float(static_cast<uint32_t>(stg_ptr[jj * 64 + 32 + lane]) << 16);
+            const float s = sigmoid_f(g);
+            const float x = v[jj];
+            const uint16_t dg = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(x * u * s * (1.0f + g * (1.0f - s)))) : uint16_t(0);
+            const uint16_t du = ok ? __bfloat16_as_ushort(__float2bfloat16_rn(x * g * s)) : uint16_t(0);
+            stg_ptr[jj * 64 + lane] = dg;
+            stg_ptr[jj * 64 + 32 + lane] = du;
           }
           __syncwarp();
           const int fb = tl.ft * kTileF + q * 32;
@@ -990,6 +1004,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             }
           }
           __syncwarp();
+          if (c0 + 16 < tl.width) prefetch_gu(tl, c0 + 16);
         } else {
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj)
@@ -1016,6 +1031,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         else mbar_arrive(acc_empty(pipes ? (it & 1) : 0));
       }
     }
+    // A staged chunk prefetched for a tile that was then abandoned lands
+    // before the CTA can exit.
+    if constexpr (kGuStaged) cp_async_wait<0>();
   }
 
   tc_fence_before();
