@@ -407,9 +407,13 @@ def _launches_per_step(cfg):
     # copy (with the adapter the adapter kernels gather the rows instead).
     words = (cfg.T + 31) // 32
     route = 2 if words <= 32 and words * cfg.E <= 8192 else (3 if cfg.adapter else 4)
+    # a forward GEMM runs as two launches (experts of at most 192 rows on the
+    # narrow kernel, the rest on the wide one) once the mean expert holds more
+    # than 96 rows
+    per_gemm = 2 if cfg.T * cfg.k > 96 * cfg.E else 1
     if not cfg.swiglu:
-        return route + 1
-    n = route + 2 + 1                           # gate/up, down, combine
+        return route + per_gemm
+    n = route + 2 * per_gemm + 1                # gate/up, down, combine
     if cfg.adapter:
         n += 1                                  # adapter apply
     if cfg.train:

@@ -160,7 +160,7 @@ int choose_bn(int64_t M, int E, int max_bn) {
   }
   // 1.5x the mean rows per expert, so that most experts fit one token tile
   // (their weights are streamed once); experts with more rows are split by
-  // the kernel into equal tiles of at most BN rows.
+  // the kernel into tiles of BN rows and a shorter last one.
   const double mean = static_cast<double>(M) / std::max(1, E);
   const double want = std::max(1.0, 1.5 * mean);
   const int bn = static_cast<int>((std::min(want, static_cast<double>(max_bn)) + 15.0) / 16.0) * 16;
@@ -189,6 +189,10 @@ moe_status check_groups(const moe_groups* g, int E) {
   if (g->E != E) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
+
+// Experts with more rows than this run the wide-tile forward when the layer
+// is large enough to split by size (moe_grouped_qgemm_fwd).
+constexpr int kWideMinRows = 192;
 
 struct GemmPlan {
   int BN, stages, a_stages, grid, n_ftiles, acc_cols, tmem_cols, n_issuers, lanes, dq_warps;
@@ -221,7 +225,7 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   // weights are then dequantized for half as many token tiles, which pays for
   // the shallower ring (measured at 341 rows per expert: -12 % and -21 % on
   // the two backward GEMMs; at 85 rows wider tiles only cost stages).
-  pl.BN = choose_bn(M, w->E, pl.pair ? 192 : 96);
+  pl.BN = choose_bn(M, w->E, pl.pair ? 192 : (mode == kModeFwdW ? 2 * kWideHalfRows : 96));
   if (mode == kModeBwd && !getenv("MOEQ_BN") && M >= 128 * static_cast<int64_t>(w->E))
     pl.BN = 192;
   if (pl.pair) pl.BN = (pl.BN + 31) / 32 * 32;   // pair MMAs take N in steps of 32
@@ -262,7 +266,20 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   auto fits = [&](int s, int sa) {
     return static_cast<int>(s * pl.stage_bytes + gemm_fixed_smem_bytes(mode, s, sa, w->E)) <= avail;
   };
-  if (mode != kModeBwd) {
+  if (mode == kModeFwdW) {
+    // Wide token tiles: one issuer and one accumulator of up to 384 columns;
+    // the rest of tensor memory holds A stages of 32 columns (64-wide fills),
+    // a multiple of the two lanes.
+    pl.lanes = 2;
+    pl.dq_warps = 16;
+    pl.n_issuers = 1;
+    pl.halves = false;
+    pl.a_stages = std::min(8, (512 - pl.acc_cols) / 32 / 2 * 2);
+    pl.tmem_cols = 512;
+    int stages = 16;
+    while (stages > 2 && !fits(stages, pl.a_stages)) stages -= 2;
+    pl.stages = stages;
+  } else if (mode != kModeBwd) {
     // A stage of a 128-wide fill: 64 tensor-memory columns. The most issuers
     // that still leave four A stages; with two issuers and wide accumulators
     // (more than 128 columns each) two A stages, handed over in halves, so
@@ -356,51 +373,55 @@ moe_status check_workspace(void* ws, size_t* ws_bytes, size_t need) {
 // Runs one grouped GEMM launch over the rows of `bmat` (a, a' or dout).
 moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qweight* w,
                     const moe_groups* g, void* out, int64_t ldo, void* saved, const GemmPlan& pl,
-                    cudaStream_t s, const int32_t* b_rows = nullptr) {
-  const int F = (mode == kModeFwd) ? (epi == MOE_EPI_SWIGLU ? w->N / 2 : w->N) : w->K;
-  const int R = (mode == kModeFwd) ? w->K : w->N;
+                    cudaStream_t s, const int32_t* b_rows = nullptr, int32_t m_lo = 0,
+                    int32_t m_hi = 0x7fffffff) {
+  const bool fwd = gemm_is_fwd(mode);
+  const int F = fwd ? (epi == MOE_EPI_SWIGLU ? w->N / 2 : w->N) : w->K;
+  const int R = fwd ? w->K : w->N;
+  const uint32_t fill = (mode == kModeFwd || mode == kModeBwdT) ? 128 : 64;   // reduction per fill
   CUtensorMap tb, tw, ts;
   const bool int4 = w->fmt == MOE_W_INT4_G32_BF16;
   const uint64_t esz = int4 ? 2 : 1;
   const CUtensorMapDataType sdt = int4 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t E = w->E, N = w->N, K = w->K;
-  const uint32_t chunks = (mode == kModeBwd) ? 1 : 2;      // 64-element K chunks per fill
+  const uint32_t chunks = fill / 64;                        // 64-element K chunks per fill
   {  // token rows: [M][R] BF16 viewed as (64, M, R/64) -> smem [chunk][BN rows][64]
+     // (wide tiles: two boxes of kWideHalfRows rows)
     const uint64_t dims[3] = {64, static_cast<uint64_t>(M), static_cast<uint64_t>(R) / 64};
     const uint64_t strides[2] = {static_cast<uint64_t>(R) * 2, 128};
-    const uint32_t box[3] = {64, static_cast<uint32_t>(pl.pair ? pl.BN / 2 : pl.BN), chunks};
+    const uint32_t rows = (mode == kModeFwdW) ? kWideHalfRows : (pl.pair ? pl.BN / 2 : pl.BN);
+    const uint32_t box[3] = {64, rows, chunks};
     if (!make_map_3d(&tb, bmat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return MOE_ERR_CUDA;
   }
-  if (mode == kModeFwd && epi == MOE_EPI_SWIGLU) {
+  // Forward packed rows: fill / 2 bytes a row, 64-byte or 32-byte swizzle.
+  const CUtensorMapSwizzle wsw = (fill == 128) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (fwd && epi == MOE_EPI_SWIGLU) {
     // packed [E][N][K/2] as [2E][N/2][K/2]: one box brings 64 gate and the 64 up rows
     const uint64_t wd[3] = {K / 2, N / 2, 2 * E};
     const uint64_t ws[2] = {K / 2, (N / 2) * (K / 2)};
-    const uint32_t wb[3] = {64, 64, 2};
-    // scales [E][K/32][N] as [E*K/32][2][N/2] -> smem [4 groups][2 halves][64]
+    const uint32_t wb[3] = {fill / 2, 64, 2};
+    // scales [E][K/32][N] as [E*K/32][2][N/2] -> smem [groups][2 halves][64]
     const uint64_t sd[3] = {N / 2, 2, E * (K / 32)};
     const uint64_t ss[2] = {(N / 2) * esz, N * esz};
-    const uint32_t sb[3] = {64, 2, 4};
-    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb,
-                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+    const uint32_t sb[3] = {64, 2, fill / 32};
+    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb, wsw) ||
         !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
-  } else if (mode == kModeFwd) {
+  } else if (fwd) {
     const uint64_t wd[3] = {K / 2, E * N, 1};
     const uint64_t ws[2] = {K / 2, E * N * (K / 2)};
-    const uint32_t wb[3] = {64, 128, 1};
+    const uint32_t wb[3] = {fill / 2, 128, 1};
     const uint64_t sd[3] = {N, E * (K / 32), 1};
     const uint64_t ss[2] = {N * esz, E * (K / 32) * N * esz};
-    const uint32_t sb[3] = {128, 4, 1};
-    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb,
-                     CU_TENSOR_MAP_SWIZZLE_64B) ||
+    const uint32_t sb[3] = {128, fill / 32, 1};
+    if (!make_map_3d(&tw, w->packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, wd, ws, wb, wsw) ||
         !make_map_3d(&ts, w->scales, sdt, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return MOE_ERR_CUDA;
   } else {
     // backward: one box is the fill's reduction rows n (64, or 128 with A in
     // tensor memory) x the tile's 128 features (64 B); scales [4 groups][rows]
-    const uint32_t fill = (mode == kModeBwdT) ? 128 : 64;
     const uint64_t wd[3] = {K / 2, E * N, 1};
     const uint64_t ws[2] = {K / 2, E * N * (K / 2)};
     const uint32_t wb[3] = {64, fill, 1};
@@ -432,6 +453,12 @@ moe_status run_gemm(int mode, int epi, const void* bmat, int64_t M, const moe_qw
   p.stage_bytes = pl.stage_bytes;
   p.pipes = pl.pipes ? 1 : 0;
   p.a_halves = pl.halves ? 1 : 0;
+  // Token tiles of an expert: equal widths; MOEQ_SPLIT=bn gives BN-row tiles
+  // and a shorter last one (fewer padding rows, measured no faster; tuning).
+  p.split_even = 1;
+  if (const char* env = getenv("MOEQ_SPLIT")) p.split_even = (strcmp(env, "bn") == 0) ? 0 : 1;
+  p.m_lo = m_lo;
+  p.m_hi = m_hi;
   // Gathered rows: the token-row tensor map above is encoded (over the same
   // base) but not read; the producers copy row b_rows[p] of bmat instead.
   p.b_rows = b_rows;
@@ -595,7 +622,21 @@ moe_status moe_grouped_qgemm_fwd(const void* a, const int32_t* a_rows, int64_t M
   if (epi != MOE_EPI_NONE && epi != MOE_EPI_SWIGLU) return MOE_ERR_INVALID_ARG;
   if (epi == MOE_EPI_SWIGLU && w->N % 128 != 0) return MOE_ERR_UNSUPPORTED;
   const int F = (epi == MOE_EPI_SWIGLU) ? w->N / 2 : w->N;
-  const GemmPlan pl = plan_gemm(kModeFwd, M, w, F, epi == MOE_EPI_SWIGLU ? 64 : 128, w->fmt);
+  // Experts with more than kWideMinRows rows run the wide-tile kernel (token
+  // tiles of up to 384 rows, so each weight is dequantized once per 384 rows
+  // of an expert instead of once per 96), the rest the narrow one: two
+  // launches over the same active list, each taking one size class, once the
+  // mean expert holds more than 96 rows (below that few experts are that
+  // large, and the extra launch would cost more than it saves). MOEQ_WIDE=0
+  // keeps every expert narrow, MOEQ_WIDE=1 makes every expert wide (tuning).
+  // Not with gathered rows or CTA pairs.
+  int wide_mode = (M > 96 * static_cast<int64_t>(w->E)) ? 2 : 0;   // 0 narrow, 1 wide, 2 both
+  if (const char* env = getenv("MOEQ_WIDE")) wide_mode = (atoi(env) == 1) ? 1 : 0;
+  if (const char* env = getenv("MOEQ_PAIR")) if (atoi(env) == 1) wide_mode = 0;
+  if (a_rows && !adapter) wide_mode = 0;   // the wide kernel reads its rows by tensor map only
+  const int tile_f = epi == MOE_EPI_SWIGLU ? 64 : 128;
+  const GemmPlan pl = plan_gemm(wide_mode == 1 ? kModeFwdW : kModeFwd, M, w, F, tile_f, w->fmt);
+  const GemmPlan plw = (wide_mode == 2) ? plan_gemm(kModeFwdW, M, w, F, tile_f, w->fmt) : pl;
   const size_t need = adapter ? align_up(static_cast<size_t>(M) * w->K * 2, 256) : 0;
   if ((st = check_workspace(ws, ws_bytes, need)) != MOE_OK) return st;
   if (!ws && ws_bytes) return MOE_OK;   // size query
@@ -613,9 +654,16 @@ moe_status moe_grouped_qgemm_fwd(const void* a, const int32_t* a_rows, int64_t M
     cudaError_t e = launch_adapter_apply(a, a_rows, adapter, g->expert_offsets, w->E,
                                          static_cast<int>(M), w->K, xa, s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    return run_gemm(kModeFwd, epi, xa, M, w, g, out, F, saved_gu, pl, s);
+    a = xa;
   }
-  return run_gemm(kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s, a_rows);
+  const int32_t* rows = adapter ? nullptr : a_rows;
+  if (wide_mode == 2) {
+    st = run_gemm(kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s, rows, 0, kWideMinRows);
+    if (st != MOE_OK) return st;
+    return run_gemm(kModeFwdW, epi, a, M, w, g, out, F, saved_gu, plw, s, rows, kWideMinRows + 1);
+  }
+  return run_gemm(wide_mode == 1 ? kModeFwdW : kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s,
+                  rows);
 }
 
 moe_status moe_grouped_qgemm_bwd_dx(const void* dout, int64_t M, const moe_qweight* w,

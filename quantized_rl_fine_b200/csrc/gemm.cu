@@ -58,6 +58,7 @@ constexpr int kTileF = 128;            // output features per tile (MMA M)
 constexpr uint32_t kABytes = kTileF * 64 * 2;   // 16 KiB dequantized A tile (backward fill)
 constexpr uint32_t kStageBytesEpi = 2048;       // epilogue staging block per warp
 constexpr uint32_t kScratchBytes = 1024;        // kModeBwdT transpose scratch per dequant warp
+constexpr int kWideHalf = kWideHalfRows;        // kModeFwdW: token rows of a tile's first MMA
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -105,9 +106,10 @@ struct Tile {
 
 // Tile t of the tile list: active index a with tile_start[a] <= t (shared
 // memory), then feature tile major, token tile minor inside the expert. An
-// expert's m rows are split into nrt = ceil(m / BN) token tiles of equal width
-// (ceil(m / nrt) rounded up to kRound, 16, or 32 for CTA-pair MMAs), so the
-// MMAs run on few padding rows.
+// expert's m rows make nrt = ceil(m / BN) token tiles: BN rows each and a last
+// tile with the rest, rounded up to kRound (16, or 32 for CTA-pair MMAs), so
+// only that last tile runs padding rows (p.split_even: nrt tiles of equal
+// width ceil(m / nrt) rounded up to kRound instead).
 template <int kRound>
 __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* tile_start, int A,
                                             int t) {
@@ -123,16 +125,24 @@ __device__ __forceinline__ Tile decode_tile(const GemmArgs& p, const int32_t* ti
   const int seg1 = p.offsets[r.e + 1];
   const int m = seg1 - seg0;
   const int nrt = (m + p.BN - 1) / p.BN;
-  r.width = (((m + nrt - 1) / nrt) + kRound - 1) & ~(kRound - 1);
   r.ft = local / nrt;
-  r.row0 = seg0 + (local - r.ft * nrt) * r.width;
+  const int tt = local - r.ft * nrt;
+  if (p.split_even) {
+    r.width = (((m + nrt - 1) / nrt) + kRound - 1) & ~(kRound - 1);
+    r.row0 = seg0 + tt * r.width;
+  } else {
+    const int rows = (tt + 1 < nrt) ? p.BN : m - (nrt - 1) * p.BN;
+    r.width = (rows + kRound - 1) & ~(kRound - 1);
+    r.row0 = seg0 + tt * p.BN;
+  }
   r.row_end = min(seg1, r.row0 + r.width);
   return r;
 }
 
 // Every CTA builds the tile list of the launch in shared memory:
 // tile_start[a] = sum over active experts a' < a of n_ftiles * ceil(m_e / BN),
-// tile_start[A] = total. Offsets that do not describe M rows give an empty
+// tile_start[A] = total, counting only experts with m_lo <= m_e <= m_hi (the
+// others get no tiles: a launch can take one size class of experts). Offsets that do not describe M rows give an empty
 // list and raise the device error. Returns A (0 when inconsistent).
 __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* warp_tot) {
   const int nthr = blockDim.x;
@@ -154,7 +164,7 @@ __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* 
   for (int a = a0; a < a1; ++a) {
     const int e = p.active[a];
     const int m = p.offsets[e + 1] - p.offsets[e];
-    local += p.n_ftiles * ((m + p.BN - 1) / p.BN);
+    if (m >= p.m_lo && m <= p.m_hi) local += p.n_ftiles * ((m + p.BN - 1) / p.BN);
   }
   const int lane = tid & 31, w = tid >> 5, nw = nthr >> 5;
   int x = local;
@@ -172,7 +182,7 @@ __device__ int build_tile_list(const GemmArgs& p, int32_t* tile_start, int32_t* 
     tile_start[a] = run;
     const int e = p.active[a];
     const int m = p.offsets[e + 1] - p.offsets[e];
-    run += p.n_ftiles * ((m + p.BN - 1) / p.BN);
+    if (m >= p.m_lo && m <= p.m_hi) run += p.n_ftiles * ((m + p.BN - 1) / p.BN);
   }
   if (tid == nthr - 1) {
     int total = 0;
@@ -207,17 +217,28 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   // loads and dequantizes its own weight rows and loads half of the token
   // rows (forward only).
   static_assert(!PAIR || MODE == kModeFwd, "CTA pairs run the forward kernels");
+  // kModeFwdW: token tiles of up to 2 x kWideHalf rows, each K step issued as
+  // two MMAs (tile columns [0, kWideHalf) and the rest) into one accumulator;
+  // 64-wide fills, so an A stage is 32 tensor-memory columns.
+  constexpr bool kWide = (MODE == kModeFwdW);
+  constexpr bool kFwd = gemm_is_fwd(MODE);
+  static_assert(!kWide || (!PAIR && LANES == 2), "wide tiles run on single CTAs with two lanes");
   constexpr int kWRound = PAIR ? 32 : 16;
   constexpr uint32_t kScEl = (FMT == MOE_W_INT4_G32_BF16) ? 2 : 1;
-  constexpr bool kGluRows = (MODE == kModeFwd && EPI == MOE_EPI_SWIGLU);
+  constexpr bool kGluRows = (kFwd && EPI == MOE_EPI_SWIGLU);
   // Forward and kModeBwdT: fills of 128 reduction elements; the dequantized
   // A tile goes to tensor memory (64 columns per fill). kModeBwd: fills of
   // 64, A in a 128B-swizzled MN-major shared-memory tile.
   constexpr bool kTmemA = (MODE != kModeBwd);
-  constexpr int kFillK = kTmemA ? 128 : 64;
+  constexpr int kFillK = (kTmemA && !kWide) ? 128 : 64;
+  constexpr int kFillGroups = kFillK / 32;                        // quantization groups per fill row
+  constexpr int kAStageCols = kFillK / 2;                         // tensor-memory columns of an A stage
   constexpr uint32_t kSmemA = kTmemA ? 0u : kABytes;
-  constexpr uint32_t kWqFill = kTmemA ? 8192u : 4096u;            // packed bytes per fill
-  constexpr uint32_t kScFill = (kTmemA ? 512u : 256u) * kScEl;    // scale bytes per fill
+  // Packed and scale bytes per fill: 128 weight rows x kFillK elements
+  // (forward: kFillK / 2 bytes and kFillK / 32 scales a row), or kFillK
+  // reduction rows x 128 features (backward: 64 bytes and 4 scales a row).
+  constexpr uint32_t kWqFill = 64u * kFillK;
+  constexpr uint32_t kScFill = 4u * kFillK * kScEl;
   constexpr int kBChunks = kFillK / 64;                           // 128-byte K chunks of B
 
   extern __shared__ uint8_t smem_raw[];
@@ -229,7 +250,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const uint32_t stage_bytes = p.stage_bytes;
   // One [rows][64] BF16 chunk of token rows; a pair's CTAs hold BN / 2 rows each.
   const uint32_t b_chunk = static_cast<uint32_t>(PAIR ? p.BN / 2 : p.BN) * 128u;
-  const uint32_t b_bytes = b_chunk * kBChunks;
+  // (wide tiles: always two boxes of kWideHalf rows)
+  const uint32_t b_bytes = kWide ? 2u * kWideHalf * 128u : b_chunk * kBChunks;
   // One stage: [B kBChunks x BN*128][A 16 KiB (backward only)][packed][scales]
   auto B_at = [&](int s) { return base + s * stage_bytes; };
   auto A_at = [&](int s) { return base + s * stage_bytes + b_bytes; };
@@ -481,16 +503,23 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           if (!mbar_wait(empty(st), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t bar = full_tma(st);
           mbar_arrive_expect_tx(bar, tx);
-          tma_load_3d_hint(B_at(st), &tm_b, bar, 0, brow, kb * kBChunks, pol_b);
-          if constexpr (MODE == kModeFwd) {
+          if constexpr (kWide) {
+            // token rows in two boxes of kWideHalf rows: [2 x kWideHalf][64]
+            tma_load_3d_hint(B_at(st), &tm_b, bar, 0, brow, kb, pol_b);
+            tma_load_3d_hint(B_at(st) + kWideHalf * 128u, &tm_b, bar, 0, brow + kWideHalf, kb, pol_b);
+          } else {
+            tma_load_3d_hint(B_at(st), &tm_b, bar, 0, brow, kb * kBChunks, pol_b);
+          }
+          if constexpr (kFwd) {
+            // kFillK / 2 packed bytes and kFillGroups scales per weight row
             if constexpr (EPI == MOE_EPI_SWIGLU) {
-              // packed: [2 halves][64 rows][64 B]; scales: [4 groups][2 halves][64]
-              tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * 64, tl.ft * 64, 2 * tl.e, pol_w);
-              tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * 64, 0, tl.e * (K / 32) + kb * 4, pol_w);
+              // packed: [2 halves][64 rows][kFillK / 2 B]; scales: [groups][2 halves][64]
+              tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * (kFillK / 2), tl.ft * 64, 2 * tl.e, pol_w);
+              tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * 64, 0, tl.e * (K / 32) + kb * kFillGroups, pol_w);
             } else {
-              // packed: [128 rows][64 B]; scales: [4 groups][128 rows]
-              tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * 64, tl.e * N + tl.ft * kTileF, 0, pol_w);
-              tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * kTileF, tl.e * (K / 32) + kb * 4, 0, pol_w);
+              // packed: [128 rows][kFillK / 2 B]; scales: [groups][128 rows]
+              tma_load_3d_hint(W_at(st), &tm_wq, bar, kb * (kFillK / 2), tl.e * N + tl.ft * kTileF, 0, pol_w);
+              tma_load_3d_hint(S_at(st), &tm_sc, bar, tl.ft * kTileF, tl.e * (K / 32) + kb * kFillGroups, 0, pol_w);
             }
           } else {
             // packed: [64 rows][64 B]; scales: [4 groups][64 rows]
@@ -579,8 +608,13 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           kbs = 1;
         }
         const int q_acc = pipes ? j : 0;       // accumulator handoff barriers of this tile
-        const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kTileF : kTileF, tile_at(t).width,
+        const int width = tile_at(t).width;
+        // Wide tiles: columns [0, kWideHalf) and [kWideHalf, width) as two MMAs.
+        const int n2 = kWide ? width - kWideHalf : 0;
+        const uint32_t idesc = idesc_bf16_f32(PAIR ? 2 * kTileF : kTileF,
+                                              (kWide && n2 > 0) ? kWideHalf : width,
                                               MODE == kModeBwd ? 1u : 0u, 0u);
+        const uint32_t idesc2 = idesc_bf16_f32(kTileF, n2 > 0 ? n2 : 16, 0u, 0u);
         if (!wait_x(acc_empty(q_acc), static_cast<uint32_t>(it & 1) ^ 1u)) { ok = false; break; }
         tc_fence_after();
         uint32_t acc = 0;
@@ -618,7 +652,20 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
             tc_fence_after();
             const uint64_t b0 = smem_desc_sw128(B_at(st), 16, 1024);
             if (elect_one()) {
-              if constexpr (kTmemA) {
+              if constexpr (kWide) {
+                // A stage sa: 128 lanes x 32 columns (64 K); each K step of 16
+                // (8 columns) multiplies the tile's first kWideHalf token rows
+                // and, for wider tiles, the rest into accumulator columns
+                // kWideHalf onward.
+                const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * kAStageCols);
+                const uint64_t b1 = b0 + ((kWideHalf * 128u) >> 4);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                  const uint32_t accum = (ks == 0) ? acc : 1u;
+                  mma_ts(d_tmem, a0 + 8 * ks, b0 + 2 * ks, idesc, accum);
+                  if (n2 > 0) mma_ts(d_tmem + kWideHalf, a0 + 8 * ks, b1 + 2 * ks, idesc2, accum);
+                }
+              } else if constexpr (kTmemA) {
                 // A stage st: 128 lanes x 64 columns (two BF16 per column): K=16 = 8 columns.
                 const uint32_t a0 = tmem_base + a_col0 + static_cast<uint32_t>(sa * 64);
                 const uint64_t b1 = b0 + (b_chunk >> 4);
@@ -707,13 +754,14 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
         if (!mbar_wait(full_tma(cur), cur_ph, abort_flag)) { ok = false; break; }
         const uint32_t wq = W_at(cur);
         const uint32_t sc = S_at(cur);
-        if constexpr (MODE == kModeFwd) {
-          // Packed rows are 64 bytes with the TMA 64-byte swizzle (16-byte chunk
-          // index ^= (row >> 1) & 3). Scales: [4 groups][128 rows].
-          const uint32_t prow = wq + src * 64;
-          const uint32_t sw = (src >> 1) & 3;
+        if constexpr (kFwd) {
+          // Packed rows are kFillK / 2 bytes with the TMA swizzle of that width
+          // (16-byte chunk index ^= (row >> 1) & 3 for 64-byte rows, ^= (row >> 2)
+          // & 1 for 32-byte rows). Scales: [kFillGroups groups][128 rows].
+          const uint32_t prow = wq + src * (kFillK / 2);
+          const uint32_t sw = (kFillK == 128) ? ((src >> 1) & 3) : ((src >> 2) & 1);
           const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + a_col0 +
-                                static_cast<uint32_t>(cur_a * 64);
+                                static_cast<uint32_t>(cur_a * kAStageCols);
           // The A stage (or, with halves, each half of it) must have been
           // released by the MMAs of the fill that used it SA fills ago. A
           // warp covers the fill's four 32-element groups (one warp per lane
@@ -724,7 +772,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           // k), which keeps only 16 results live. A half past the reduction
           // length (K % 128 == 64) is written as zeros, so neither the
           // zero-filled codes nor a foreign scale can reach the MMA.
-          constexpr int kGroups = 4 / kParts;
+          constexpr int kGroups = kFillGroups / kParts;
           const int units = (halves && kParts == 1) ? 2 : 1;
           for (int u = 0; u < units && ok; ++u) {
             const int half = (kParts == 2) ? hk : u;
@@ -735,7 +783,7 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
               const int c = hk * kGroups + cc;
               if (units == 2 && (c >> 1) != half) continue;
               uint32_t o[16];
-              if (kb_cur * kFillK + (c >> 1) * 64 >= p.R) {
+              if (kb_cur * kFillK + c * 32 >= p.R) {
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
               } else {
@@ -1130,6 +1178,18 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_w
   MOEQ_CASE_SINGLE(kModeBwd, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU_BWD)
   MOEQ_CASE_SINGLE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
   MOEQ_CASE_SINGLE(kModeBwd, MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU_BWD)
+  if (mode == kModeFwdW) {
+    // one plan only: two lanes of eight dequant warps each, single CTAs
+    if (pair || lanes != 2 || dq_warps != 16) return cudaErrorInvalidValue;
+#define MOEQ_WIDE(F_, E_) \
+    if (fmt == F_ && epi == E_) return launch_grouped_qgemm_t<kModeFwdW, F_, E_, 2, 0, 16>(tb, tw, ts, p, grid, smem, s);
+    MOEQ_WIDE(MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
+    MOEQ_WIDE(MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU)
+    MOEQ_WIDE(MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
+    MOEQ_WIDE(MOE_W_MXFP4_G32_E8M0, MOE_EPI_SWIGLU)
+#undef MOEQ_WIDE
+    return cudaErrorInvalidValue;
+  }
   MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_INT4_G32_BF16, MOE_EPI_NONE)
   MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_INT4_G32_BF16, MOE_EPI_SWIGLU_BWD)
   MOEQ_CASE_SINGLE(kModeBwdT, MOE_W_MXFP4_G32_E8M0, MOE_EPI_NONE)
@@ -1143,7 +1203,9 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_w
 uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair) {
   const uint32_t el = (fmt == MOE_W_INT4_G32_BF16) ? 2u : 1u;
   uint32_t b;
-  if (mode != kModeBwd)   // B 2 chunks (BN / 2 rows in a pair), packed 128 rows x 64 B, scales 4 x 128
+  if (mode == kModeFwdW)  // B 2 boxes of kWideHalf rows x 1 chunk, packed 128 rows x 32 B, scales 2 x 128
+    b = 2u * kWideHalf * 128u + 4096u + 256u * el;
+  else if (mode != kModeBwd)   // B 2 chunks (BN / 2 rows in a pair), packed 128 rows x 64 B, scales 4 x 128
     b = static_cast<uint32_t>(pair ? BN / 2 : BN) * 256u + 8192u + 512u * el;
   else                    // B 1 chunk, A 16 KiB, packed 64 rows x 64 B, scales 4 x 64
     b = static_cast<uint32_t>(BN) * 128u + kABytes + 4096u + 256u * el;

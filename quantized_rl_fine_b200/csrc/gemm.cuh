@@ -11,6 +11,10 @@ namespace moeq {
 constexpr int kModeFwd = 0;    // D[f, t] = sum_k W[e][f][k] a[t][k]
 constexpr int kModeBwd = 1;    // D[f, t] = sum_n W[e][n][f] dout[t][n], A in shared memory
 constexpr int kModeBwdT = 2;   // the same, A in tensor memory (128-wide fills, transposed dequant)
+constexpr int kModeFwdW = 3;   // forward with wide token tiles (up to 384 rows: two MMAs per
+                               // K step), 64-wide fills, one accumulator
+__host__ __device__ constexpr bool gemm_is_fwd(int mode) { return mode == kModeFwd || mode == kModeFwdW; }
+constexpr int kWideHalfRows = 192;   // kModeFwdW: token rows of a tile's first MMA (and TMA box)
 
 struct GemmArgs {
   const int32_t* offsets;     // [E+1] expert row offsets
@@ -31,6 +35,9 @@ struct GemmArgs {
   uint32_t stage_bytes;       // bytes of one stage (1 KiB multiple)
   int32_t pipes;              // 1: two tile pipelines (two issuers, each accumulating whole tiles)
   int32_t a_halves;           // forward: 1 = each A stage handed over in two 64-wide halves
+  int32_t split_even;         // 1: an expert's token tiles have equal widths; 0: BN-row tiles
+                              // and a shorter last one
+  int32_t m_lo, m_hi;         // only experts with m_lo <= rows <= m_hi get tiles in this launch
   __nv_bfloat16* out;         // [M][ldo]
   int64_t ldo;
   __nv_bfloat16* saved;       // fwd SwiGLU: written [M][N]; bwd SwiGLU: read [M][2K]

@@ -73,6 +73,11 @@ def test_step_accounting_of_a_training_step_with_adapter():
     # routing (3), adapter (gathers the rows), gate/up, down, combine, scatter
     # of dy, two backward GEMMs, fused adapter backward, combine of dx
     (C.TRAIN_INT4, 12),
+    # top-k, scan, scatter, row copy, gate/up and down as two launches each
+    # (narrow and wide experts: 341 rows per expert on average), combine
+    (C.TRILLION_INT4.with_(T=16384), 9),
+    # the same for the Zipf-routed MXFP4 layer (256 rows per expert on average)
+    (C.ZIPF_MXFP4, 9),
 ])
 def test_launch_count_per_step(cfg, kernels):
     assert bench._launches_per_step(cfg) == kernels

@@ -29,6 +29,14 @@ RAGGED_MX = MoEConfig("ragged_mxfp4", E=5, k=3, d=128, f=192, T=37, fmt="mxfp4",
 # of 160 or more rows per expert), wider than any forward tile.
 WIDE = MoEConfig("wide_int4", E=4, k=2, d=256, f=256, T=300, fmt="int4", swiglu=True,
                  logits="normal", adapter=True, train=True, seed=2003)
+# More than 128 rows per expert: the forward takes the wide-tile plan (one
+# token tile of up to 384 rows per expert, two MMAs per K step past 192 rows).
+# About 256 rows per expert (one tile each, 192 + 64 columns), and about 500
+# (two tiles, 384 + the rest), MXFP4 with a 192-long down reduction.
+WIDE_FWD = MoEConfig("wide_fwd_int4", E=4, k=2, d=256, f=256, T=512, fmt="int4", swiglu=True,
+                     logits="normal", adapter=True, train=True, seed=2004)
+WIDE_MX = MoEConfig("wide_fwd_mxfp4", E=2, k=1, d=128, f=192, T=1000, fmt="mxfp4", swiglu=True,
+                    logits="normal", adapter=False, train=True, seed=2005)
 
 
 def _to(wl, dev):
@@ -375,4 +383,49 @@ def test_shared_memory_backward_matches_the_oracle(monkeypatch, cfg):
     rows per expert on) against the oracle."""
     monkeypatch.setenv("MOEQ_BWD_SMEM_A", "1")
     _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, RAGGED_MX, WIDE], ids=["int4", "mxfp4_ragged", "wide_int4"])
+def test_even_token_tile_split_matches_the_oracle(monkeypatch, cfg):
+    """An expert's rows go to token tiles of BN rows and a shorter last one by
+    default; this runs the equal-width split (every tile ceil(m / nrt) rows
+    rounded up to 16) against the oracle."""
+    monkeypatch.setenv("MOEQ_SPLIT", "even")
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [WIDE_FWD, WIDE_MX], ids=["int4_256_rows", "mxfp4_500_rows"])
+def test_wide_token_tile_forward_matches_the_oracle(cfg):
+    """The planned wide-tile forward (more than 128 rows per expert): token
+    tiles of up to 384 rows, two MMAs per K step past 192 rows, 64-wide fills
+    with 32-column A stages, one accumulator."""
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [TINY_TRAIN, RAGGED_MX, WIDE], ids=["int4", "mxfp4_ragged", "wide_int4"])
+def test_forced_wide_plan_matches_the_oracle(monkeypatch, cfg):
+    """The wide-tile forward forced on small shapes (token tiles of 16 to 240
+    rows, one MMA per K step below 193 rows)."""
+    monkeypatch.setenv("MOEQ_WIDE", "1")
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
+@pytest.mark.parametrize("cfg", [WIDE_FWD, WIDE_MX], ids=["int4_256_rows", "mxfp4_500_rows"])
+def test_wide_and_narrow_forward_give_the_same_bits(monkeypatch, cfg):
+    """Every plan accumulates a token's column in the same K order, one MMA
+    column per token: the wide-tile forward and the narrow one (96-row tiles,
+    two tile pipelines) give bit-identical outputs."""
+    wl = _gpu_workload(cfg)
+    outs = []
+    for env in ("1", "0"):
+        monkeypatch.setenv("MOEQ_WIDE", env)
+        st = layer.forward(wl["x"], wl["logits"], wl["w_gu"], wl["w_d"], cfg.k, cfg.chunk_size,
+                           adapter=wl.get("adapter"), train=cfg.train)
+        outs.append((st["h"].clone(), st["y"].clone(), st["saved_gu"].clone()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
