@@ -225,7 +225,14 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
   // weights are then dequantized for half as many token tiles, which pays for
   // the shallower ring (measured at 341 rows per expert: -12 % and -21 % on
   // the two backward GEMMs; at 85 rows wider tiles only cost stages).
-  pl.BN = choose_bn(M, w->E, pl.pair ? 192 : (mode == kModeFwdW ? 2 * kWideHalfRows : 96));
+  // Wide tiles: up to 384 rows (MOEQ_WIDE_BN caps them lower, tuning).
+  int wide_cap = 2 * kWideHalfRows;
+  if (const char* env = getenv("MOEQ_WIDE_BN")) {
+    const int v = atoi(env);
+    if (v >= 16 && v <= 2 * kWideHalfRows && v % 16 == 0) wide_cap = v;
+  }
+  pl.BN = choose_bn(M, w->E, pl.pair ? 192 : (mode == kModeFwdW ? wide_cap : 96));
+  if (mode == kModeFwdW) pl.BN = std::min(pl.BN, wide_cap);
   if (mode == kModeBwd && !getenv("MOEQ_BN") && M >= 128 * static_cast<int64_t>(w->E))
     pl.BN = 192;
   if (pl.pair) pl.BN = (pl.BN + 31) / 32 * 32;   // pair MMAs take N in steps of 32
@@ -267,14 +274,15 @@ GemmPlan plan_gemm(int mode, int64_t M, const moe_qweight* w, int F, int tile_f,
     return static_cast<int>(s * pl.stage_bytes + gemm_fixed_smem_bytes(mode, s, sa, w->E)) <= avail;
   };
   if (mode == kModeFwdW) {
-    // Wide token tiles: one issuer and one accumulator of up to 384 columns;
-    // the rest of tensor memory holds A stages of 32 columns (64-wide fills),
-    // a multiple of the two lanes.
+    // Wide token tiles: A stages of 32 columns (64-wide fills), a multiple of
+    // the two lanes, next to one accumulator of up to 384 columns, or to two
+    // (two issuers, two tile pipelines) while two accumulators and four A
+    // stages fit (tiles of at most 192 rows).
     pl.lanes = 2;
     pl.dq_warps = 16;
-    pl.n_issuers = 1;
+    pl.n_issuers = (2 * pl.acc_cols + 4 * 32 <= 512) ? 2 : 1;
     pl.halves = false;
-    pl.a_stages = std::min(8, (512 - pl.acc_cols) / 32 / 2 * 2);
+    pl.a_stages = std::min(8, (512 - pl.n_issuers * pl.acc_cols) / 32 / 2 * 2);
     pl.tmem_cols = 512;
     int stages = 16;
     while (stages > 2 && !fits(stages, pl.a_stages)) stages -= 2;

@@ -250,8 +250,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   const uint32_t stage_bytes = p.stage_bytes;
   // One [rows][64] BF16 chunk of token rows; a pair's CTAs hold BN / 2 rows each.
   const uint32_t b_chunk = static_cast<uint32_t>(PAIR ? p.BN / 2 : p.BN) * 128u;
-  // (wide tiles: always two boxes of kWideHalf rows)
-  const uint32_t b_bytes = kWide ? 2u * kWideHalf * 128u : b_chunk * kBChunks;
+  // (wide tiles: one box of kWideHalf rows, two when tiles may be wider)
+  const bool wide2 = kWide && p.BN > kWideHalf;
+  const uint32_t b_bytes = kWide ? (wide2 ? 2u : 1u) * kWideHalf * 128u : b_chunk * kBChunks;
   // One stage: [B kBChunks x BN*128][A 16 KiB (backward only)][packed][scales]
   auto B_at = [&](int s) { return base + s * stage_bytes; };
   auto A_at = [&](int s) { return base + s * stage_bytes + b_bytes; };
@@ -324,7 +325,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     }
     mbar_init(acc_full(0), pipes ? 1 : p.n_issuers);
     mbar_init(acc_full(1), 1);
-    mbar_init(acc_empty(0), PAIR ? 8 : 4);
+    // (wide tiles with one accumulator: the four epilogue warps and every
+    // dequant warp drain it)
+    mbar_init(acc_empty(0), PAIR ? 8 : ((kWide && p.n_issuers == 1) ? 4 + kDqWarps : 4));
     mbar_init(acc_empty(1), PAIR ? 8 : 4);
     mbar_init(drain_bar, p.n_issuers);
     *abort_flag = 0;
@@ -363,6 +366,76 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
   // Tensor-memory columns: [partial accumulator 0 .. NI-1][A stage 0 .. S-1 (forward)].
   const int NI = p.n_issuers;
   const uint32_t a_col0 = static_cast<uint32_t>(NI * p.acc_cols);
+  // Wide tiles with one accumulator: no MMA can start while a tile's
+  // accumulator drains, and the dequant warps have then run out of A stages.
+  // So the tile's 16-column chunks are shared by the five warps of each lane
+  // quarter, its epilogue warp (helper 0) and its four dequant warps (helpers
+  // 1-4, by index in the quarter): chunk i goes to helper i % 5. Each helper
+  // stores its results straight from registers (a row's 16 or 32 values per
+  // store instruction are contiguous), without the staging block.
+  const bool helpers = kWide && NI == 1;
+  constexpr int kHelpers = 1 + kDqWarps / 4;
+  auto wide_chunk = [&](const Tile& tl, int c0) {
+    const int qq = warp & 3;
+    float v[16];
+    {
+      uint32_t ua[16];
+      tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(qq * 32) << 16) + static_cast<uint32_t>(c0), ua);
+      tmem_wait_ld();
+#pragma unroll
+      for (int jj = 0; jj < 16; ++jj) v[jj] = __uint_as_float(ua[jj]);
+    }
+    const int nrows = min(16, tl.row_end - (tl.row0 + c0));
+    uint16_t* out16 = reinterpret_cast<uint16_t*>(p.out);
+    if constexpr (kGluRows) {
+      // lanes 0-15: gate values of features pr, lanes 16-31: their up values
+      const int pr = lane & 15;
+      const bool is_gate = lane < 16;
+      const int hrow0 = is_gate ? 0 : 8;
+      const int fcol = tl.ft * 64 + qq * 16 + pr;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        const float mine = is_gate ? v[jj] : v[jj + 8];
+        const float got = __shfl_xor_sync(0xffffffffu, is_gate ? v[jj + 8] : v[jj], 16);
+        const float g = is_gate ? mine : got;
+        const float u = is_gate ? got : mine;
+        const uint16_t h = __bfloat16_as_ushort(__float2bfloat16_rn(silu_f(g) * u));
+        if (hrow0 + jj < nrows)
+          out16[static_cast<int64_t>(tl.row0 + c0 + hrow0 + jj) * p.ldo + fcol] = h;
+      }
+      if (p.saved) {
+        uint16_t* sv16 = reinterpret_cast<uint16_t*>(p.saved);
+        const int scol = is_gate ? fcol : N / 2 + fcol;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)
+          if (jj < nrows)
+            sv16[static_cast<int64_t>(tl.row0 + c0 + jj) * N + scol] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
+      }
+    } else {
+      const int f = tl.ft * kTileF + qq * 32 + lane;
+      if (f < p.F) {
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)
+          if (jj < nrows)
+            out16[static_cast<int64_t>(tl.row0 + c0 + jj) * p.ldo + f] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(v[jj]));
+      }
+    }
+  };
+  // Helper h's share of tile tl's epilogue (the tile is the CTA's it-th).
+  auto wide_epilogue = [&](const Tile& tl, int it, int h) {
+    // lane 0's result decides for the warp, so the tensor-memory loads below
+    // (warp-collective) run on all lanes or none
+    const bool r = mbar_wait(acc_full(0), static_cast<uint32_t>(it & 1), abort_flag);
+    if (!__shfl_sync(0xffffffffu, r ? 1 : 0, 0)) return false;
+    tc_fence_after();
+    for (int c0 = 16 * h; c0 < tl.width; c0 += 16 * kHelpers) wide_chunk(tl, c0);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty(0));
+    return true;
+  };
 
   if (warp < kProdWarps && gather) {
     // ------------------------------------------------------------ gathering producers
@@ -506,7 +579,8 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           if constexpr (kWide) {
             // token rows in two boxes of kWideHalf rows: [2 x kWideHalf][64]
             tma_load_3d_hint(B_at(st), &tm_b, bar, 0, brow, kb, pol_b);
-            tma_load_3d_hint(B_at(st) + kWideHalf * 128u, &tm_b, bar, 0, brow + kWideHalf, kb, pol_b);
+            if (wide2)
+              tma_load_3d_hint(B_at(st) + kWideHalf * 128u, &tm_b, bar, 0, brow + kWideHalf, kb, pol_b);
           } else {
             tma_load_3d_hint(B_at(st), &tm_b, bar, 0, brow, kb * kBChunks, pol_b);
           }
@@ -895,6 +969,9 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
           if (lane == 0) mbar_arrive(full_a(cur_a));
         }
       }
+      // Wide tiles: this warp's share of the tile's epilogue, once its MMAs
+      // are done (every dequant warp arrives on the accumulator's barrier).
+      if (helpers && ok) ok = wide_epilogue(tile_at(t), li, 1 + ((warp - kDqWarp0) >> 2));
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
@@ -935,6 +1012,10 @@ grouped_qgemm_kernel(const __grid_constant__ CUtensorMap tm_b,
     int r0 = 0;                             // (first fill of the tile) % NI
     for (int t = t_first; t < total; t += t_step, ++it) {
       const Tile tl = tile_at(t);
+      if (helpers) {                        // wide tiles: helper 0's share of the chunks
+        if (!wide_epilogue(tl, it, 0)) break;
+        continue;
+      }
       if constexpr (kGuStaged) prefetch_gu(tl, 0);
       // Issuer j wrote its partial in this tile iff one of the tile's nkb
       // fills f has f % NI == j. With tile pipelines the tile's whole sum is
@@ -1203,8 +1284,8 @@ cudaError_t launch_grouped_qgemm(int mode, int fmt, int epi, int lanes, int dq_w
 uint32_t gemm_stage_bytes(int mode, int BN, int fmt, bool pair) {
   const uint32_t el = (fmt == MOE_W_INT4_G32_BF16) ? 2u : 1u;
   uint32_t b;
-  if (mode == kModeFwdW)  // B 2 boxes of kWideHalf rows x 1 chunk, packed 128 rows x 32 B, scales 2 x 128
-    b = 2u * kWideHalf * 128u + 4096u + 256u * el;
+  if (mode == kModeFwdW)  // B 1 or 2 boxes of kWideHalf rows x 1 chunk, packed 128 rows x 32 B, scales 2 x 128
+    b = (BN > kWideHalf ? 2u : 1u) * kWideHalf * 128u + 4096u + 256u * el;
   else if (mode != kModeBwd)   // B 2 chunks (BN / 2 rows in a pair), packed 128 rows x 64 B, scales 4 x 128
     b = static_cast<uint32_t>(pair ? BN / 2 : BN) * 256u + 8192u + 512u * el;
   else                    // B 1 chunk, A 16 KiB, packed 64 rows x 64 B, scales 4 x 64
