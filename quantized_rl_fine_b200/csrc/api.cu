@@ -666,9 +666,15 @@ moe_status moe_grouped_qgemm_fwd(const void* a, const int32_t* a_rows, int64_t M
   }
   const int32_t* rows = adapter ? nullptr : a_rows;
   if (wide_mode == 2) {
-    st = run_gemm(kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s, rows, 0, kWideMinRows);
+    // MOEQ_WIDE_MIN moves the size-class cut (tuning).
+    int cut = kWideMinRows;
+    if (const char* env = getenv("MOEQ_WIDE_MIN")) {
+      const int v = atoi(env);
+      if (v >= 16 && v <= 2 * kWideHalfRows) cut = v;
+    }
+    st = run_gemm(kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s, rows, 0, cut);
     if (st != MOE_OK) return st;
-    return run_gemm(kModeFwdW, epi, a, M, w, g, out, F, saved_gu, plw, s, rows, kWideMinRows + 1);
+    return run_gemm(kModeFwdW, epi, a, M, w, g, out, F, saved_gu, plw, s, rows, cut + 1);
   }
   return run_gemm(wide_mode == 1 ? kModeFwdW : kModeFwd, epi, a, M, w, g, out, F, saved_gu, pl, s,
                   rows);
