@@ -414,6 +414,17 @@ def test_forced_wide_plan_matches_the_oracle(monkeypatch, cfg):
     assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
 
 
+@pytest.mark.parametrize("cfg", [RAGGED_MX, WIDE], ids=["mxfp4_ragged", "wide_int4"])
+def test_forced_wide_plan_without_tile_pipelines_matches_the_oracle(monkeypatch, cfg):
+    """The wide-tile forward with two issuers taking every other fill into
+    partial accumulators (no tile pipelines; token rows and weights share the
+    shared-memory stages)."""
+    monkeypatch.setenv("MOEQ_WIDE", "1")
+    monkeypatch.setenv("MOEQ_PIPES", "0")
+    _run_layer_and_compare(cfg)
+    assert moeq.moe_get_device_error() == moeq.DEVERR_NONE
+
+
 @pytest.mark.parametrize("cfg", [WIDE_FWD, WIDE_MX], ids=["int4_256_rows", "mxfp4_500_rows"])
 def test_wide_and_narrow_forward_give_the_same_bits(monkeypatch, cfg):
     """Every plan accumulates a token's column in the same K order, one MMA
