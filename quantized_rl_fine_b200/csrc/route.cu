@@ -17,8 +17,10 @@
 //     with shared-memory atomicOr; the rank of token t inside expert e is the
 //     popcount of the mask below t, which gives the stable position
 //     offsets[e] + block_base[e] + rank.
-//  4. permute_rows_kernel: one warp per permuted row copies its token row
-//     with 16-byte loads and stores across the whole grid.
+//  4. permute_rows_kernel: one warp per token reads its row once, with
+//     16-byte loads, and writes it to each of its k permuted rows. (One warp
+//     per permuted row reads every token row k times; at 16384 tokens x 14 KB
+//     those re-reads miss L2 and cost as much DRAM traffic as the writes.)
 // Small launches (T <= 1024 and a token-by-expert bit matrix of at most 8192
 // words) replace steps 2 and 3 by route_tail_kernel: one block builds, for
 // every expert, the bit mask of its tokens over all T, and takes counts,
@@ -327,26 +329,38 @@ route_scatter_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __rest
   }
 }
 
-// One warp per permuted row p: x_perm[p] = x[perm_token[p]] (16-byte moves).
+// One warp per token t: x_perm[inv_perm[t * k + j]] = x[t] for j < k
+// (16-byte moves; the row is read once).
 __global__ void __launch_bounds__(256)
-permute_rows_kernel(const int32_t* __restrict__ perm_token, int M, const uint4* __restrict__ x,
+permute_rows_kernel(const int32_t* __restrict__ inv_perm, int T, int k, const uint4* __restrict__ x,
                     uint4* __restrict__ x_perm, int64_t row_vec) {
   grid_dependency_wait();
   grid_dependents_launch();
-  const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (p >= M) return;
-  const uint4* src = x + static_cast<int64_t>(perm_token[p]) * row_vec;
-  uint4* dst = x_perm + static_cast<int64_t>(p) * row_vec;
-  int64_t c = lane;
-  for (; c + 96 < row_vec; c += 128) {
-    const uint4 a0 = src[c], a1 = src[c + 32], a2 = src[c + 64], a3 = src[c + 96];
-    dst[c] = a0;
-    dst[c + 32] = a1;
-    dst[c + 64] = a2;
-    dst[c + 96] = a3;
+  if (t >= T) return;
+  // Lane j < k holds the permuted row of (t, j); k <= 32.
+  const int64_t my_dst =
+      (lane < k) ? static_cast<int64_t>(__ldg(inv_perm + static_cast<int64_t>(t) * k + lane)) * row_vec : 0;
+  const uint4* src = x + static_cast<int64_t>(t) * row_vec;
+  // 128 16-byte units of the row per step (four a lane); the loops stay
+  // warp-uniform around the shuffles, and units past the row are skipped.
+  for (int64_t base = 0; base < row_vec; base += 128) {
+    uint4 a[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t c = base + lane + 32 * u;
+      a[u] = (c < row_vec) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+    }
+    for (int j = 0; j < k; ++j) {
+      const int64_t dst = __shfl_sync(0xffffffffu, my_dst, j);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t c = base + lane + 32 * u;
+        if (c < row_vec) x_perm[dst + c] = a[u];
+      }
+    }
   }
-  for (; c < row_vec; c += 32) dst[c] = src[c];
 }
 
 }  // namespace
@@ -446,9 +460,8 @@ cudaError_t launch_route(const float* logits, const void* x, int T, int E, int k
                      static_cast<const int32_t*>(offsets), T, E, k, perm_token, inv_perm);
   }
   if (err != cudaSuccess || x == nullptr) return err;
-  const int M = T * k;
-  return launch_pdl(permute_rows_kernel, dim3((M + 7) / 8), dim3(256), 0, s,
-                    static_cast<const int32_t*>(perm_token), M, static_cast<const uint4*>(x),
+  return launch_pdl(permute_rows_kernel, dim3((T + 7) / 8), dim3(256), 0, s,
+                    static_cast<const int32_t*>(inv_perm), T, k, static_cast<const uint4*>(x),
                     static_cast<uint4*>(x_perm), d / 8);
 }
 
