@@ -248,7 +248,10 @@ adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restric
       const int64_t gi = static_cast<int64_t>(pr) * K + 32 * b + 8 * ch;
       const int64_t xi = (rows ? static_cast<int64_t>(__ldg(rows + pr)) : pr) * K + 32 * b + 8 * ch;
       vx[h] = ok ? __ldg(reinterpret_cast<const uint4*>(x + xi)) : make_uint4(0, 0, 0, 0);
-      vg[h] = ok ? __ldg(reinterpret_cast<const uint4*>(dxp + gi)) : make_uint4(0, 0, 0, 0);
+      // dx' is read once and dx written once: streaming (evict-first) hints
+      // on both (measured at the training shape, 384 experts x 85 rows:
+      // 446 -> 415 us)
+      vg[h] = ok ? __ldcs(reinterpret_cast<const uint4*>(dxp + gi)) : make_uint4(0, 0, 0, 0);
     }
     __syncwarp();                        // the previous step's stores from xs are done
 #pragma unroll
@@ -314,8 +317,8 @@ adapter_bwd_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restric
     for (int h = 0; h < 4; ++h) {
       const int idx = lane + 32 * h, row = idx >> 2, ch = idx & 3;
       if (c0 + row < p1)
-        *reinterpret_cast<uint4*>(dx + static_cast<int64_t>(c0 + row) * K + 32 * b + 8 * ch) =
-            *reinterpret_cast<const uint4*>(&xs[warp][row][8 * ch]);
+        __stcs(reinterpret_cast<uint4*>(dx + static_cast<int64_t>(c0 + row) * K + 32 * b + 8 * ch),
+               *reinterpret_cast<const uint4*>(&xs[warp][row][8 * ch]));
     }
   }
   float* dst = dR + (static_cast<int64_t>(e) * nb + b) * 1024;
