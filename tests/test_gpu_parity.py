@@ -124,6 +124,19 @@ def test_route_permute_bit_exact(T, E, k, C):
     _check_routing(r, logits, x, k, C, E)
 
 
+@pytest.mark.parametrize("T,E,k,d", [(1500, 64, 4, 1032), (2048, 128, 8, 8)])
+def test_route_permute_copies_rows_of_any_width(T, E, k, d):
+    # More than 1024 tokens: the histogram path and its row copy (one warp per
+    # token, 128 16-byte units a step), with a ragged last step (129 units)
+    # and with a single unit per row.
+    g = torch.Generator().manual_seed(T + d)
+    logits = torch.randn((T, E), generator=g)
+    x = torch.randn((T, d), generator=g).to(torch.bfloat16)
+    r = moeq.moe_route_permute(logits.to(DEV), x.to(DEV), k, 8)
+    torch.cuda.synchronize()
+    _check_routing(r, logits, x, k, 8, E)
+
+
 def test_route_uniform_logits_full_size():
     wl = _gpu_workload(MXFP4_UP)
     r = moeq.moe_route_permute(wl["logits"], wl["x"], MXFP4_UP.k, MXFP4_UP.chunk_size)
